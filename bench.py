@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the MISA routed indexer on B200: scored (query, prefix-token) pairs per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+pool keys -> route heads -> routed token scoring + top-k (config 4 adds the
+MISA-dagger re-rank).  Default workload: 128K prefill, H=32 indexer heads,
+pool block 128, m=8 routed heads, top-k 2048 (every query scores its whole
+causal prefix: 8.59e9 pairs per step).  Inputs are larger than L2 (q alone is
+1.07 GB), so no L2 flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs an independent problem of the same
+shape on its own GPU (weak scaling, no data-path collective); the step time
+is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle as it stands on this host's cores on a
+bounded sample of the same workload (the oracle is the only reference: the
+pages publish no code).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "scored query x prefix-token pairs/sec (MISA routed indexer)"
+UNIT = "pairs/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d["bf16_tflops_sustained"], source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def score_src_sha():
+    h = hashlib.sha256()
+    for f in ("score.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "long_context_sparse_misa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_pair(kernel: str, workload: str):
+    """DRAM bytes per scored pair from a committed ncu summary whose kernel
+    source hash matches the current source; None otherwise."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    sha = score_src_sha()
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith(".md"):
+            continue
+        with open(os.path.join(pdir, fn)) as f:
+            text = f.read()
+        m_k = re.search(r"^kernel:\s*(\S+)", text, re.M)
+        m_w = re.search(r"^workload:\s*(\S+)", text, re.M)
+        m_s = re.search(r"^source_sha:\s*(\S+)", text, re.M)
+        m_t = re.search(r"^dram_bytes_per_pair:\s*([0-9.eE+-]+)", text, re.M)
+        if m_k and m_w and m_s and m_t and m_k.group(1) == kernel and \
+                m_w.group(1) == workload and m_s.group(1) == sha:
+            return float(m_t.group(1))
+    return None
+
+
+class Clocks:
+    """Samples nvidia-smi every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid, self.proc, self.lines = uuid, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_init():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_config(wl, cfg):
+    from misa_synth import CONFIGS
+    c = CONFIGS[cfg]
+    return {"workload": c["name"], "seqs": c["S"], "prefix_len": c["L"], "queries": wl.T,
+            "H": c["H"], "d": c["d"], "pool_block": c["B"], "m": c["m"], "k": c["k"],
+            "k_cand": c["k_cand"] or None, "pairs_per_step": wl.pairs,
+            "l2": "inputs larger than L2 (126 MB): no flush" if wl.q_bits.nbytes + wl.K_bits.nbytes > 2 * 126e6
+                  else "L2 flushed between steps (256 MB write)"}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def cpu_oracle_sample(wl, budget_s, seed=0):
+    import numpy as np
+    import oracle
+    try:
+        import threadpoolctl
+        cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    Kf = oracle.widen_bf16(wl.K_bits)
+    t0 = time.perf_counter()
+    Kbar = oracle.pool_keys(Kf, wl.key_offsets, wl.B)
+    t_pool = time.perf_counter() - t0
+    boff = oracle.block_offsets(wl.key_offsets, wl.B)
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(wl.T)
+    qs = wl.q_seq
+    pairs, rows, t_rows = 0, 0, 0.0
+    for i in order:
+        s = int(qs[i])
+        k0, k1 = int(wl.key_offsets[s]), int(wl.key_offsets[s + 1])
+        t1 = time.perf_counter()
+        res = oracle.misa_query(oracle.widen_bf16(wl.q_bits[i]), wl.w[i].astype(np.float64),
+                                Kf[k0:k1], Kbar[boff[s]:boff[s + 1]], int(wl.q_pos[i]), wl.B,
+                                wl.m, wl.k_cand or wl.k)
+        if wl.k_cand:
+            oracle.hier_rerank_query(oracle.widen_bf16(wl.q_bits[i]),
+                                     wl.w[i].astype(np.float64), Kf[k0:k1], res["idx"], wl.k)
+        t_rows += time.perf_counter() - t1
+        pairs += int(wl.q_pos[i]) + 1
+        rows += 1
+        if t_rows > budget_s:
+            break
+    # pooling is per step; charge the sample its share
+    t = t_rows + t_pool * pairs / max(wl.pairs, 1)
+    return {"value": pairs / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {wl.T} query rows (random, seed {seed}), {pairs} pairs, "
+                      f"{t:.2f} s incl. pro-rated pooling; numpy fp64"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from misa_synth import make_config
+    wl = make_config(args.config)
+    per_step = max(1.0, 60.0 / max(args.steps + args.warmup, 1))
+    for s in range(args.warmup):
+        cpu_oracle_sample(wl, per_step / 4, seed=100 + s)
+    vals, pairs_total, t_total, last = [], 0, 0.0, None
+    for s in range(args.steps):
+        last = cpu_oracle_sample(wl, per_step, seed=s)
+        vals.append(last["value"])
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl.pairs / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, args.config), "impl": "reference",
+            "cpu_baseline": {k: last[k] for k in ("kind", "cores", "sample")} | {"value": value,
+                                                                               "unit": UNIT},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "note": "CPU oracle (numpy fp64) on a bounded sample per step; ms_per_step is the "
+                    "pairs/s-extrapolated time of a full step"}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import long_context_sparse_misa_b200 as misa
+    from misa_synth import make_config
+
+    world, rank, local = dist_init()
+    cfg = args.config
+    wl = make_config(cfg, seed=1000 + cfg + 100 * rank)
+    hier = bool(wl.k_cand)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    prob = misa.Problem.from_workload(wl, device=dev)
+    K = torch.from_numpy(wl.K_bits).to(dev)
+    q = torch.from_numpy(wl.q_bits).to(dev)
+    w = torch.from_numpy(wl.w).to(dev)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k, k_cand=wl.k_cand, device=dev)
+    run = (lambda: ix.hier(q, w, K)) if hier else (lambda: ix.misa(q, w, K))
+    small_inputs = wl.q_bits.nbytes + wl.K_bits.nbytes < 2 * 126e6
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small_inputs else None
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        run()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    code, bits = misa.stream_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits}) after warm-up")
+
+    # ---- timed region (device time, CUDA events, max over ranks)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = Clocks(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    torch.cuda.synchronize()
+    barrier(world)
+    misa.profile_enable(True)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    code, bits = misa.stream_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits}) in the timed region")
+    ms_step = ms / args.steps
+    pairs = wl.pairs
+    value = pairs * world / (ms_step / 1e3)
+
+    # ---- roofline of the dominant kernel (routed scoring on tcgen05)
+    peaks = load_peaks()
+    kname = "score"
+    k_ms, k_launch = prof.get(kname, (float("nan"), 0))
+    flops = 2.0 * wl.m * wl.d * pairs * args.steps
+    achieved = flops / (k_ms / 1e3) / 1e12
+    tpp = traffic_per_pair(kname, workload_config(wl, cfg)["workload"])
+    launches_per_step = k_launch / args.steps
+    roofline = {"kernel": "score_kernel (tcgen05 routed scoring)", "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_sustained"],
+                "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                "algorithmic_flops_per_launch": 2.0 * wl.m * wl.d * pairs / max(launches_per_step, 1),
+                "launches_per_step": launches_per_step,
+                "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
+    kernels = {n: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps,
+                   "share": t / max(sum(v[0] for v in prof.values()), 1e-9)}
+               for n, (t, c) in prof.items()}
+    gpu_launches = sum(c for _, c in prof.values())
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 q,k with 1% planted needles; "
+                    "w ~ N(0,1)/sqrt(H) fp32)",
+            "config": workload_config(wl, cfg) | {"parallelism": f"independent problem per GPU x{world}"},
+            "latency_ms": ms_step, "roofline": roofline, "kernels": kernels,
+            "gpu_launches": gpu_launches, "clocks": clk}
+
+    # ---- dense DSA indexer on the same inputs (the in-run comparison)
+    if not args.no_dense:
+        dense_steps = max(1, min(args.steps, 5))
+        for _ in range(1):
+            if flush is not None:
+                flush.fill_(1)
+            ix.dense(q, w, K)
+        torch.cuda.synchronize()
+        barrier(world)
+        misa.profile_enable(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(dense_steps):
+            if flush is not None:
+                flush.fill_(1)
+            ix.dense(q, w, K)
+        e1.record()
+        torch.cuda.synchronize()
+        dprof = misa.profile_collect()
+        misa.profile_enable(False)
+        dms = max_over_ranks(e0.elapsed_time(e1), world) / dense_steps
+        d_k_ms = dprof.get("score", (float("nan"), 0))[0] / dense_steps
+        d_flops = 2.0 * wl.H * wl.d * pairs
+        line["dense_dsa"] = {"ms_per_step": dms, "value": pairs * world / (dms / 1e3),
+                             "unit": UNIT, "misa_speedup": dms / ms_step,
+                             "score_kernel_tflops": d_flops / (d_k_ms / 1e3) / 1e12,
+                             "score_kernel_frac": d_flops / (d_k_ms / 1e3) / 1e12 / peaks["bf16_sustained"]}
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(a).pin_memory()
+        K_h, q_h, w_h = pin(wl.K_bits), pin(wl.q_bits), pin(wl.w)
+        idx_h = torch.empty(tuple(ix.idx.shape), dtype=torch.int32).pin_memory()
+        val_h = torch.empty(tuple(ix.val.shape), dtype=torch.float32).pin_memory()
+        e2e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            K.copy_(K_h, non_blocking=True)
+            q.copy_(q_h, non_blocking=True)
+            w.copy_(w_h, non_blocking=True)
+            run()
+            idx_h.copy_(ix.idx, non_blocking=True)
+            val_h.copy_(ix.val, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+        line["e2e"] = {"value": pairs * world / (ems / 1e3), "unit": UNIT,
+                       "ms_per_step": ems,
+                       "h2d_bytes_per_step": K_h.nbytes + q_h.nbytes + w_h.nbytes,
+                       "d2h_bytes_per_step": idx_h.nbytes + val_h.nbytes}
+
+    # ---- CPU oracle on this host, rank 0 at N=1
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(wl, args.cpu_budget_s)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

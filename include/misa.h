@@ -1,0 +1,181 @@
+/*
+ * misa.h -- C ABI of the MISA routed sparse-attention indexer for NVIDIA B200 (sm_100a).
+ *
+ * Method: "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
+ * Inference" (Zhou et al., 2026).  The DSA indexer scores every prefix token
+ * of a query with all H indexer heads,
+ *     I[t,s] = sum_h w[t,h] * ReLU(q[t,h] . k[s]),   keys s = 0..t,
+ * and keeps the top-k tokens for the main attention.  MISA treats the H heads
+ * as a mixture-of-experts pool: a router on mean-pooled key blocks keeps m
+ * heads per query, and only those m heads run the token-level scoring.
+ * MISA-dagger keeps k_cand routed candidates and re-ranks them with all H heads.
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory.  Scratch space is the caller's workspace
+ *     (size from misa_workspace_size).
+ *   - bf16 tensors are passed as uint16_t bit patterns.  Rows are row-major
+ *     and 16-byte aligned; head_dim must be 128.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return code reports argument and launch errors
+ *     only.  Device-side conditions (a bounded wait that timed out, an index
+ *     out of range, a position or candidate out of its sequence) set bits in
+ *     a per-device status word read by misa_stream_status.
+ *   - No call throws; on error the message is kept in a thread-local buffer
+ *     (misa_last_error_string).
+ *   - Ties: heads are ranked by (router score desc, head index asc); tokens by
+ *     (score desc, token index asc); -0 counts as +0.  A query whose prefix is
+ *     shorter than k selects every prefix token and pads its row with index
+ *     -1 and value -inf.  Row order of idx/val is unspecified.
+ */
+#ifndef MISA_H_
+#define MISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* misa_stream_t; /* cudaStream_t */
+
+/* Return codes. */
+enum {
+  MISA_OK = 0,
+  MISA_ERR_INVALID_ARG = 1,        /* null pointer, bad size, misaligned pointer */
+  MISA_ERR_UNSUPPORTED = 2,        /* valid but not built: head_dim != 128, m not a power of two ... */
+  MISA_ERR_WORKSPACE_TOO_SMALL = 3,
+  MISA_ERR_CUDA = 4,               /* a CUDA runtime call failed (message has the CUDA error) */
+  MISA_ERR_DEVICE_TIMEOUT = 5,     /* misa_stream_status only */
+  MISA_ERR_DEVICE_BOUNDS = 6,      /* misa_stream_status only */
+  MISA_ERR_DEVICE_BAD_INPUT = 7    /* misa_stream_status only */
+};
+
+/* Bits of the device status word. */
+#define MISA_STATUS_TIMEOUT   0x1u /* a bounded wait in a kernel gave up; that CTA returned early */
+#define MISA_STATUS_BOUNDS    0x2u /* an index fell outside its buffer; the access was skipped */
+#define MISA_STATUS_BAD_INPUT 0x4u /* a query position or candidate outside its sequence, or a NaN score */
+
+/*
+ * Problem description (the shapes of one indexer call).
+ *
+ * Keys of all sequences are packed: K is [total_keys, head_dim] bf16 and
+ * sequence s owns rows key_offsets[s] .. key_offsets[s+1]-1.  Its pooled keys
+ * (one per block of `block` consecutive keys, the last block possibly
+ * partial) are rows block_offsets[s] .. block_offsets[s+1]-1 of Kbar, with
+ * block_offsets[s+1]-block_offsets[s] = ceil(L_s / block)  (gist.science
+ * summary, "Methodologie: MISA": M = ceil(L/B) blocks).  Queries of sequence
+ * s are rows query_offsets[s] .. query_offsets[s+1]-1 of q / w; query t sits
+ * at position q_pos[t] in its sequence and sees keys 0..q_pos[t] (causal,
+ * self included).
+ */
+typedef struct {
+  int32_t num_seqs;              /* S >= 1 */
+  int32_t num_queries;           /* T >= 0 */
+  int32_t num_heads;             /* H, 1..64 */
+  int32_t head_dim;              /* d, must be 128 */
+  int32_t block;                 /* B, pooling block, 1..4096 */
+  int32_t max_seq_len;           /* host-side upper bound on every L_s (sizes grids) */
+  int64_t total_keys;            /* rows of K = key_offsets[S] */
+  int64_t total_blocks;          /* rows of Kbar = block_offsets[S] */
+  const int64_t* key_offsets;    /* device [S+1], non-decreasing, key_offsets[0] = 0 */
+  const int64_t* block_offsets;  /* device [S+1], see misa_block_offsets */
+  const int32_t* query_offsets;  /* device [S+1], non-decreasing, query_offsets[0] = 0 */
+  const int32_t* q_pos;          /* device [T], 0 <= q_pos[t] < L_seq(t) */
+} misa_problem_t;
+
+/* Bytes of workspace that any entry point below needs for this problem with
+ * m routed heads, final top-k `k` and MISA-dagger candidate count `k_cand`
+ * (0 if unused).  Returns 0 on invalid arguments. */
+size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_t k_cand);
+
+/* block_offsets[s] = sum_{s'<s} ceil(L_s' / block) from key_offsets
+ * (device arrays, S+1 entries each). */
+int misa_block_offsets(const int64_t* key_offsets, int32_t num_seqs, int32_t block,
+                       int64_t* block_offsets, misa_stream_t stream);
+
+/* Step 1 -- mean-pooled keys (gist.science summary, "Methodologie: MISA",
+ * Lightweight Block-Pooled Router: mean-pooled indexer keys per block).
+ * Kbar[b,:] = (1/|b|) sum_{s in b} K[s,:], the last block of a sequence
+ * averaged over the keys present.  Summed in fp64, divided in fp64, rounded
+ * once to fp32.
+ *   K    [total_keys, 128] bf16;  Kbar [total_blocks, 128] fp32 (written). */
+int misa_pool_keys(const misa_problem_t* p, const uint16_t* K, float* Kbar, misa_stream_t stream);
+
+/* Step 2 -- block-pooled router (same passage: per-head affinities on the
+ * pooled keys, aggregated into one importance score per head, top-h heads).
+ *     r[t,h] = w[t,h] * sum_{b < M_t} ReLU(q[t,h] . Kbar_t[b]),  M_t = ceil((t+1)/B)
+ * over the floor((t+1)/B) full blocks of Kbar plus, when (t+1) mod B != 0,
+ * the causal partial block (mean of keys floor((t+1)/B)*B .. t).  Keeps the
+ * m best heads per query.
+ *   q [T, H, 128] bf16;  w [T, H] fp32;  K, Kbar as above;  1 <= m <= H, m a power of two.
+ *   heads [T, m] int32  (written; rank order);
+ *   q_r   [T, m, 128] bf16 (written; q_r[t,j] = q[t, heads[t,j]]);
+ *   w_r   [T, m] fp32  (written; w_r[t,j] = w[t, heads[t,j]]);
+ *   router_scores [T, H] fp32 or NULL (written if not NULL). */
+int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const uint16_t* K,
+               const float* Kbar, int32_t m, int32_t* heads, uint16_t* q_r, float* w_r,
+               float* router_scores, void* ws, size_t ws_bytes, misa_stream_t stream);
+
+/* Steps 3+4 -- routed token scoring and per-query top-k (same section,
+ * Sparse Token Scoring: only the routed heads score the full prefix; the
+ * top-k tokens come from these reduced scores).
+ *     I[t,s] = sum_{j<m} w_r[t,j] * ReLU(q_r[t,j] . K[s]),  s = 0..q_pos[t]
+ *   q_r [T, m, 128] bf16;  w_r [T, m] fp32;  1 <= k <= 65536.
+ *   idx [T, k] int32 token indices within the sequence;  val [T, k] fp32 scores.
+ *   scores_dbg: NULL, or [T, scores_ld] fp32 receiving I[t, 0..q_pos[t]]
+ *   (entries past the prefix are unspecified); scores_ld >= max_seq_len. */
+int misa_score_topk(const misa_problem_t* p, const uint16_t* q_r, const float* w_r, int32_t m,
+                    const uint16_t* K, int32_t k, int32_t* idx, float* val, float* scores_dbg,
+                    int64_t scores_ld, void* ws, size_t ws_bytes, misa_stream_t stream);
+
+/* Step 5 -- MISA-dagger fine stage (gist.science summary, "Hierarchische
+ * Variant (MISA†)"): the all-head DSA indexer re-scores only the candidate
+ * tokens and keeps the final top-k.
+ *   cand [T, k_cand] int32 token indices (e.g. the idx of misa_score_topk
+ *   run with k = k_cand); entries < 0 are padding and skipped; an entry past
+ *   the query's position sets MISA_STATUS_BAD_INPUT and is skipped.
+ *   idx [T, k], val [T, k] as in misa_score_topk;  k <= k_cand <= 65536. */
+int misa_hier_rerank(const misa_problem_t* p, const uint16_t* q, const float* w,
+                     const uint16_t* K, const int32_t* cand, int32_t k_cand, int32_t k,
+                     int32_t* idx, float* val, void* ws, size_t ws_bytes, misa_stream_t stream);
+
+/* The dense DSA indexer, the in-run comparison (MISA abstract; gist.science
+ * summary, "Probleemstelling"): every head scores every prefix token.
+ *     I[t,s] = sum_{h<H} w[t,h] * ReLU(q[t,h] . K[s])
+ * Same outputs as misa_score_topk; H must be a power of two. */
+int dsa_index_dense(const misa_problem_t* p, const uint16_t* q, const float* w,
+                    const uint16_t* K, int32_t k, int32_t* idx, float* val, float* scores_dbg,
+                    int64_t scores_ld, void* ws, size_t ws_bytes, misa_stream_t stream);
+
+/* Synchronises `stream`, returns the status word of the current device in
+ * *device_status (may be NULL) and clears it.  Returns MISA_OK when the word
+ * was zero, else the MISA_ERR_DEVICE_* code of its lowest set bit;
+ * MISA_ERR_CUDA if the synchronisation itself failed. */
+int misa_stream_status(misa_stream_t stream, int32_t* device_status);
+
+/* Diagnostic: launches one CTA whose bounded wait on a barrier that nothing
+ * arrives on runs out after `wait_ms` milliseconds (1..5000); the kernel then
+ * sets MISA_STATUS_TIMEOUT and returns.  Used to test that a timed-out wait
+ * leaves the context usable.  No counterpart in the paper. */
+int misa_selftest_timeout(int32_t wait_ms, misa_stream_t stream);
+
+/* Tracing.  While enabled (on != 0), every kernel the library launches from
+ * the calling host thread is bracketed by CUDA events recorded on its launch
+ * stream.  misa_profile_collect synchronises those events and returns, per
+ * kernel name (names: max_kernels x 32 chars), the summed device time in
+ * milliseconds and the launch count, then clears the record.  Returns the
+ * number of kernel names (at most max_kernels) or a negative MISA_ERR code.
+ * No counterpart in the paper. */
+int misa_profile_enable(int32_t on);
+int misa_profile_collect(int32_t max_kernels, char* names, double* total_ms, int64_t* launches);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* misa_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MISA_H_ */

@@ -1,0 +1,89 @@
+// Host-side declarations shared by the translation units of libmisa.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/misa.h"
+
+namespace misa {
+
+constexpr int kD = 128;          // head dimension (fixed)
+constexpr int kTileKeys = 128;   // keys per MMA tile (TMEM lanes)
+constexpr int kSms = 148;
+
+// One query group: queries [q_begin, q_end) of sequence `seq`, largest position max_pos.
+// Stored as int4 {seq, q_begin, q_end, max_pos}.
+
+void set_error(const char* fmt, ...);
+int cuda_fail(cudaError_t e, const char* what);
+
+// Device status word of the current device (a __device__ variable of libmisa).
+uint32_t* status_ptr();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point: 2-D bf16
+// tensor [rows, 128] with a {64, box_rows} box and 128-byte swizzle.
+int make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
+
+int set_smem_limit(const void* kernel, int bytes);
+
+// Tracing: brackets one kernel launch with events on `st` when profiling is on.
+struct ProfScope {
+  ProfScope(const char* name, cudaStream_t st);
+  ~ProfScope();
+  int slot;
+  cudaStream_t st;
+};
+
+// ---- pool.cu
+int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* block_offsets,
+                         cudaStream_t st);
+// Build query groups of at most G queries over query rows [q_lo, q_hi).
+// groups: int4 [q_hi-q_lo + S]; count: one int.
+int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
+                       int* count, cudaStream_t st);
+int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st);
+
+// ---- route.cu
+int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, const uint16_t* K,
+                 const float* Kbar, int m, int32_t* heads, uint16_t* q_r, float* w_r,
+                 float* router_scores, const int4* groups, const int* group_count,
+                 int max_groups, int G, cudaStream_t st);
+int route_group_size(int H);
+
+// ---- score.cu
+// I[(t - q_lo) * ld + s] = sum_{j<m} wsel[t,j] ReLU(qsel[t,j] . K[key(t,s)]) for the
+// queries of the groups.  Contiguous mode (cand == nullptr): s = 0..q_pos[t].
+// Gather mode: s = slot 0..k_cand-1 of cand[t, :], key = cand[t, s].
+struct ScoreArgs {
+  const misa_problem_t* p;
+  const uint16_t* qsel;   // [T * m, 128] bf16
+  const float* wsel;      // [T, m]
+  int m;
+  const uint16_t* K;      // [total_keys, 128] bf16
+  const int32_t* cand;    // [T, k_cand] or nullptr
+  int k_cand;
+  const int4* groups;     // device group table
+  const int* group_count; // device: number of valid groups
+  int max_groups;         // host bound on the group count
+  int G;                  // queries per group
+  int q_lo;
+  float* I;               // output rows
+  int64_t ld;
+  int max_tiles;          // host bound on key tiles per group
+};
+int launch_score(const ScoreArgs& a, cudaStream_t st);
+int score_group_size(int m);
+
+// ---- topk.cu
+// For query rows [q_lo, q_hi): select the top-k of I row (t - q_lo).
+// Contiguous mode (tok == nullptr): elements 0..q_pos[t], token = element index.
+// Token mode: elements 0..n_fixed-1 with token tok[t * n_fixed + e] (< 0 = absent).
+int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32_t* tok,
+                int n_fixed, int q_lo, int q_hi, int k, int32_t* idx, float* val,
+                cudaStream_t st);
+
+}  // namespace misa

@@ -1,0 +1,402 @@
+// Token-level indexer scoring on tcgen05 tensor cores.
+//
+// Computes, for every query t of a group and key s of its causal prefix,
+//     I[t,s] = sum_{j<m} w[t,j] * ReLU(q[t,j] . k[s])
+// With the routed heads this is MISA's sparse token scoring ("MISA: Mixture
+// of Indexer Sparse Attention for Long-Context LLM Inference", gist.science
+// summary, "Methodologie: MISA", Sparse Token Scoring); with all H heads it
+// is the dense DSA indexer (abstract); in gather mode over candidate tokens
+// it is the MISA-dagger re-scoring (same page, "Hierarchische Variant").
+//
+// Layout of one CTA (one query group x a range of 128-key tiles):
+//   A operand = 128 keys x 128 dims, TMA-loaded (or cp.async-gathered) into a
+//               128-byte-swizzled K-major tile, kStages deep;
+//   B operand = the group's (query, head) rows, N = nq*m <= 256, resident;
+//   D         = TMEM, 128 lanes (one key per lane) x N fp32 columns, two
+//               buffers so the epilogue of tile i overlaps the MMAs of i+1.
+// Keys on the lanes means the head reduction of a query is a sum over m
+// adjacent columns inside one thread: the epilogue is ReLU, one FMA with the
+// head weight, and a causal compare -- no shuffles and no [m x L] tensor.
+//
+// Roles: warp 0 producer, warp 1 TMEM owner + MMA issuer (one thread),
+// warps 2..5 epilogue (TMEM lane quarter = warp % 4).
+#include "common.cuh"
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kStageBytes = kTileKeys * kD * 2;          // 32 KB: two 16 KB 64-dim halves
+constexpr int kHalfBytes = kStageBytes / 2;
+constexpr int kMaxN = 256;                               // MMA N and TMEM columns per buffer
+constexpr int kQHalfBytes = kMaxN * 128;                 // 32 KB per 64-dim half
+constexpr int kQBytes = 2 * kQHalfBytes;
+constexpr int kTmemCols = 2 * kMaxN;
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kMaxN * 4 /*w*/ +
+                           kMaxN * 4 /*pos*/ + kMaxN * 4 /*row*/ + 32 * 8 /*barriers*/ + 16;
+
+struct Smem {
+  uint8_t* q;
+  uint8_t* k;
+  float* w;
+  int* pos;
+  int* row;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* qfull;
+  uint64_t* drain;
+  uint32_t* tmem_slot;
+  int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* base =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.q = base;
+  s.k = base + kQBytes;
+  s.w = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
+  s.pos = reinterpret_cast<int*>(s.w + kMaxN);
+  s.row = s.pos + kMaxN;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.row + kMaxN);
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = s.tfull + 2;
+  s.qfull = s.tempty + 2;
+  s.drain = s.qfull + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
+  return s;
+}
+
+// All 32 lanes wait together; the outcome is warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* abort,
+                                          uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  long long t0 = 0;
+  if (lane == 0) t0 = clock64();
+  while (true) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    int give_up = 0;
+    if (lane == 0) {
+      if (*reinterpret_cast<volatile int*>(abort)) {
+        give_up = 1;
+      } else if (clock64() - t0 > kWaitCycles) {
+        *reinterpret_cast<volatile int*>(abort) = 1;
+        set_status(status, MISA_STATUS_TIMEOUT);
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+  }
+}
+
+template <int MH, bool GATHER>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                 const uint16_t* __restrict__ K, const float* __restrict__ wsel,
+                 const int32_t* __restrict__ q_pos, const int64_t* __restrict__ ko,
+                 const int32_t* __restrict__ cand, int k_cand, const int4* __restrict__ groups,
+                 const int* __restrict__ group_count, int tiles_per_split, int q_lo,
+                 float* __restrict__ I, int64_t ld, int64_t total_keys, uint32_t* status) {
+  constexpr int G = GATHER ? 1 : kMaxN / MH;
+  static_assert(G * MH <= kMaxN, "group too wide");
+  extern __shared__ uint8_t smem_raw[];
+
+  const int gi = blockIdx.x;
+  if (gi >= *group_count) return;
+  const int4 grp = groups[gi];
+  const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y, maxpos = grp.w;
+  if (maxpos < 0 || nq <= 0) return;
+  const int64_t key_base = ko[seq];
+  const int ntiles = GATHER ? (k_cand + kTileKeys - 1) / kTileKeys
+                            : (maxpos + 1 + kTileKeys - 1) / kTileKeys;
+  const int tile0 = blockIdx.y * tiles_per_split;
+  if (tile0 >= ntiles) return;
+  const int nt = min(ntiles, tile0 + tiles_per_split) - tile0;
+  const int NP = ((nq * MH + 31) / 32) * 32;  // MMA N (multiple of 32, <= 256)
+
+  Smem s = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], GATHER ? 32 : 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 4);
+    }
+    mbar_init(s.qfull, 1);
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // Per-column head weight and per-query causal limit / output row.
+    for (int c = threadIdx.x - 64; c < kMaxN; c += 128) {
+      const int qi = c / MH;
+      s.w[c] = (c < nq * MH) ? wsel[(int64_t)(qb + qi) * MH + (c - qi * MH)] : 0.f;
+    }
+    for (int qi = threadIdx.x - 64; qi < kMaxN; qi += 128) {
+      int pos = -1;
+      if (qi < nq) {
+        pos = q_pos[qb + qi];
+        const int64_t L = ko[seq + 1] - key_base;
+        if (pos < 0 || pos >= L) pos = -1;
+      }
+      s.pos[qi] = pos;
+      s.row[qi] = qb + qi - q_lo;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (!GATHER) {
+      if (lane == 0) {
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&qmap);
+        mbar_arrive_expect_tx(s.qfull, 2u * NP * 128u);
+        for (int h = 0; h < 2; ++h)
+          for (int r0 = 0; r0 < NP; r0 += 32)
+            tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
+                        qb * MH + r0);
+        int issued = 0;
+        for (int i = 0; i < nt; ++i) {
+          const int st = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          if (!mbar_wait(&s.empty[st], ph ^ 1, s.abort, status)) break;
+          mbar_arrive_expect_tx(&s.full[st], kStageBytes);
+          const int32_t krow = (int32_t)(key_base + (int64_t)(tile0 + i) * kTileKeys);
+          uint8_t* dst = s.k + st * kStageBytes;
+          tma_load_2d(&kmap, &s.full[st], dst, 0, krow);
+          tma_load_2d(&kmap, &s.full[st], dst + kHalfBytes, 64, krow);
+          issued = i + 1;
+        }
+        // Drain: the last load of every stage must have landed before the CTA exits.
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+          mbar_wait(&s.full[i % kStages], (i / kStages) & 1, s.abort, status, kDrainCycles,
+                    /*drain=*/true);
+      }
+    } else {
+      // Gather mode: rows K[key_base + cand[t, slot]] for the 128 slots of a
+      // tile; each lane copies 4 rows as 16-byte chunks into the swizzled layout.
+      const int t = qb;
+      const int pos = s.pos[0];
+      if (lane == 0) {
+        tma_prefetch_desc(&qmap);
+        mbar_arrive_expect_tx(s.qfull, 2u * NP * 128u);
+        for (int h = 0; h < 2; ++h)
+          for (int r0 = 0; r0 < NP; r0 += 32)
+            tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
+                        qb * MH + r0);
+      }
+      __syncwarp();
+      int pending = -1;  // tile whose copies are committed but not yet signalled
+      int i = 0;
+      for (; i < nt; ++i) {
+        const int st = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!warp_wait(&s.empty[st], ph ^ 1, s.abort, status)) break;
+        uint8_t* dst = s.k + st * kStageBytes;
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = lane * 4 + rr;
+          const int slot = (tile0 + i) * kTileKeys + r;
+          int tok = slot < k_cand ? cand[(int64_t)t * k_cand + slot] : -1;
+          const bool ok = tok >= 0 && tok <= pos && key_base + tok < total_keys;
+          const uint16_t* src = K + (ok ? (key_base + tok) : 0) * kD;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int half = c >> 3, cc = c & 7;
+            cp_async_16(dst + half * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4), src + c * 8,
+                        ok);
+          }
+        }
+        cp_async_commit();
+        if (pending >= 0) {
+          cp_async_wait_group<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&s.full[pending % kStages]);
+        }
+        pending = i;
+      }
+      cp_async_wait_group<0>();
+      if (pending >= 0) {
+        fence_proxy_async_smem();
+        mbar_arrive(&s.full[pending % kStages]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileKeys, NP);
+      bool ok = mbar_wait(s.qfull, 0, s.abort, status);
+      tc_fence_after();
+      const uint32_t q_addr = smem_u32(s.q);
+      for (int i = 0; ok && i < nt; ++i) {
+        const int st = i % kStages;
+        const int buf = i & 1;
+        if (!mbar_wait(&s.full[st], (i / kStages) & 1, s.abort, status)) break;
+        if (!mbar_wait(&s.tempty[buf], ((i >> 1) & 1) ^ 1, s.abort, status)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(s.k + st * kStageBytes);
+        const uint32_t d = tmem_base + buf * kMaxN;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B along K
+          const uint64_t a = sw128_kmajor_desc(k_addr + (kk >> 2) * kHalfBytes + off);
+          const uint64_t b = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes + off);
+          umma_bf16(d, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s.empty[st]);
+        umma_commit(&s.tfull[buf]);
+      }
+      // Every issued MMA must complete before TMEM is released.
+      umma_commit(s.drain);
+      mbar_wait(s.drain, 0, s.abort, status, kDrainCycles, /*drain=*/true);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int lrow = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int nchunks = NP / 32;
+    for (int i = 0; i < nt; ++i) {
+      const int buf = i & 1;
+      if (!warp_wait(&s.tfull[buf], (i >> 1) & 1, s.abort, status)) break;
+      tc_fence_after();
+      const int slot = (tile0 + i) * kTileKeys + lrow;
+      int key = slot;  // contiguous mode: token index within the sequence
+      bool key_ok = true;
+      if (GATHER) {
+        key = slot < k_cand ? cand[(int64_t)qb * k_cand + slot] : -1;
+        key_ok = key >= 0 && key <= s.pos[0] && key_base + key < total_keys;
+        if (key >= 0 && !key_ok) set_status(status, MISA_STATUS_BAD_INPUT);
+      }
+      const uint32_t taddr = lane_addr + buf * kMaxN;
+      float acc = 0.f;
+      for (int c = 0; c < nchunks; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_wait_ld();
+        if constexpr (MH <= 32) {
+          constexpr int QPC = 32 / MH;
+#pragma unroll
+          for (int qq = 0; qq < QPC; ++qq) {
+            const int qi = c * QPC + qq;
+            if (qi >= nq) break;
+            const float* wq = s.w + qi * MH;
+            float sc = 0.f;
+#pragma unroll
+            for (int j = 0; j < MH; ++j) sc = fmaf(wq[j], fmaxf(v[qq * MH + j], 0.f), sc);
+            if (GATHER) {
+              if (slot < k_cand && s.row[0] >= 0)
+                I[(int64_t)s.row[0] * ld + slot] = key_ok ? sc : -INFINITY;
+            } else if (key <= s.pos[qi]) {
+              I[(int64_t)s.row[qi] * ld + key] = sc;
+            }
+          }
+        } else {
+          constexpr int CPQ = MH / 32;
+          const int qi = c / CPQ;
+          const float* wq = s.w + c * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
+          if ((c % CPQ) == CPQ - 1) {
+            if (GATHER) {
+              if (slot < k_cand && s.row[0] >= 0)
+                I[(int64_t)s.row[0] * ld + slot] = key_ok ? acc : -INFINITY;
+            } else if (qi < nq && key <= s.pos[qi]) {
+              I[(int64_t)s.row[qi] * ld + key] = acc;
+            }
+            acc = 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int MH, bool GATHER>
+int launch_one(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap, dim3 grid,
+               int tps, cudaStream_t st) {
+  auto kern = score_kernel<MH, GATHER>;
+  int rc = set_smem_limit((const void*)kern, kSmemBytes);
+  if (rc) return rc;
+  ProfScope ps(GATHER ? "rerank_score" : "score", st);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.K, a.wsel, a.p->q_pos,
+                                          a.p->key_offsets, a.cand, a.k_cand, a.groups,
+                                          a.group_count, tps, a.q_lo, a.I, a.ld,
+                                          a.p->total_keys, status_ptr());
+  return cuda_fail(cudaGetLastError(), "score_kernel");
+}
+
+template <bool GATHER>
+int dispatch(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap, dim3 grid,
+             int tps, cudaStream_t st) {
+  switch (a.m) {
+    case 1: return launch_one<1, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 2: return launch_one<2, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 4: return launch_one<4, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 8: return launch_one<8, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 16: return launch_one<16, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 32: return launch_one<32, GATHER>(a, kmap, qmap, grid, tps, st);
+    case 64: return launch_one<64, GATHER>(a, kmap, qmap, grid, tps, st);
+    default:
+      set_error("score: head count %d is not a power of two <= 64", a.m);
+      return MISA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+int score_group_size(int m) { return kMaxN / m; }
+
+int launch_score(const ScoreArgs& a, cudaStream_t st) {
+  if (a.max_groups <= 0 || a.max_tiles <= 0) return MISA_OK;
+  CUtensorMap kmap, qmap;
+  int rc = make_kmajor_map(&kmap, a.K, a.p->total_keys, kTileKeys);
+  if (rc) return rc;
+  rc = make_kmajor_map(&qmap, a.qsel, (int64_t)a.p->num_queries * a.m, 32);
+  if (rc) return rc;
+  const int64_t work = (int64_t)a.max_groups * a.max_tiles;
+  int tps = (int)((work + 8 * kSms - 1) / (8 * kSms));
+  tps = max(1, min(tps, 64));
+  const int splits = (a.max_tiles + tps - 1) / tps;
+  if (splits > 65535) {
+    set_error("score: %d key splits exceed the grid limit", splits);
+    return MISA_ERR_UNSUPPORTED;
+  }
+  dim3 grid(a.max_groups, splits);
+  return a.cand ? dispatch<true>(a, kmap, qmap, grid, tps, st)
+                : dispatch<false>(a, kmap, qmap, grid, tps, st);
+}
+
+}  // namespace misa

@@ -1,0 +1,180 @@
+"""Agreement procedure between the CUDA indexer and the CPU oracle.
+
+Floating point: |gpu - oracle| <= ATOL + RTOL * |oracle| with ATOL = 1e-4,
+RTOL = 1e-3 (fp32 scores from bf16 inputs).  Integer results (routed head
+sets, top-k index sets) must match exactly, except entries whose oracle
+score lies within that tolerance of the m-th (heads) or k-th (tokens)
+threshold; those swaps are counted and reported.  Where the router swapped
+near-tied heads, the oracle re-scores the row with the GPU's head set, so a
+single near-tie does not spoil the whole row.  Invariants checked on every
+row: indices causal and distinct, exactly min(k, n) of them, every selected
+score >= every unselected score (up to the tolerance).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+import oracle
+
+ATOL, RTOL = 1e-4, 1e-3
+
+
+def tol(x):
+    return ATOL + RTOL * np.abs(x)
+
+
+@dataclasses.dataclass
+class Report:
+    rows: int = 0
+    head_swaps: int = 0
+    topk_swaps: int = 0
+    max_val_err: float = 0.0
+    max_r_err: float = 0.0
+    failures: list = dataclasses.field(default_factory=list)
+
+    def fail(self, msg):
+        if len(self.failures) < 20:
+            self.failures.append(msg)
+
+    def assert_ok(self):
+        assert not self.failures, "\n".join(self.failures)
+
+
+def check_heads(rep: Report, i, r_oracle, heads_gpu, m):
+    """Set compare of routed heads; returns True when the GPU set is acceptable."""
+    ref = oracle.route(r_oracle, m)
+    g = set(int(h) for h in heads_gpu)
+    o = set(int(h) for h in ref)
+    if len(g) != m or any(h < 0 or h >= len(r_oracle) for h in g):
+        rep.fail(f"row {i}: invalid head set {sorted(g)}")
+        return False
+    if g == o:
+        return True
+    thr = r_oracle[ref[-1]]
+    for h in g ^ o:
+        if abs(r_oracle[h] - thr) > tol(thr):
+            rep.fail(f"row {i}: head {h} r={r_oracle[h]:.6g} far from m-th {thr:.6g}")
+            return False
+    rep.head_swaps += 1
+    return True
+
+
+def check_topk(rep: Report, i, I_oracle, idx_gpu, val_gpu, k, tokens=None):
+    """Check one row of (idx, val) against oracle scores over `tokens`
+    (default: the prefix 0..n-1 with I_oracle indexed by token)."""
+    n = len(I_oracle)
+    if tokens is None:
+        tokens = np.arange(n)
+    score_of = dict(zip((int(t) for t in tokens), I_oracle))
+    k_eff = min(k, n)
+    sel = [int(x) for x in idx_gpu if x >= 0]
+    if len(sel) != k_eff or len(set(sel)) != k_eff:
+        rep.fail(f"row {i}: {len(sel)} selected ({len(set(sel))} distinct), expected {k_eff}")
+        return
+    if any(x not in score_of for x in sel):
+        rep.fail(f"row {i}: selected token outside the candidate/prefix set")
+        return
+    pad = [j for j, x in enumerate(idx_gpu) if x < 0]
+    if len(pad) != k - k_eff or not all(np.isneginf(val_gpu[j]) for j in pad):
+        rep.fail(f"row {i}: bad padding")
+    # values
+    sv = np.array([score_of[x] for x in sel])
+    gv = np.array([float(val_gpu[j]) for j, x in enumerate(idx_gpu) if x >= 0])
+    err = np.abs(gv - sv)
+    if len(err):
+        rep.max_val_err = max(rep.max_val_err, float((err / tol(sv)).max()))
+        if np.any(err > tol(sv)):
+            j = int(np.argmax(err - tol(sv)))
+            rep.fail(f"row {i}: value of token {sel[j]} gpu={gv[j]:.7g} oracle={sv[j]:.7g}")
+    # set compare with near-threshold allowance
+    _, ref_val = oracle.topk(np.asarray(I_oracle, dtype=np.float64), k)
+    order = np.lexsort((np.asarray(tokens), -(np.asarray(I_oracle) + 0.0)))[:k_eff]
+    ref = set(int(tokens[j]) for j in order)
+    g = set(sel)
+    if g != ref and k_eff < n:
+        thr = I_oracle[order[-1]]
+        for x in g ^ ref:
+            if abs(score_of[x] - thr) > tol(thr):
+                rep.fail(f"row {i}: token {x} I={score_of[x]:.7g} far from k-th {thr:.7g}")
+                return
+        rep.topk_swaps += len(g - ref)
+    # invariant: selected >= unselected (up to tolerance)
+    if k_eff < n:
+        unsel = np.array([v for t, v in score_of.items() if t not in g])
+        if len(unsel) and sv.min() < unsel.max() - tol(unsel.max()):
+            rep.fail(f"row {i}: selected min {sv.min():.7g} < unselected max {unsel.max():.7g}")
+
+
+def check_misa_rows(wl, rows, idx, val, heads=None, r=None, Kbar=None, k=None, m=None,
+                    rep: Report | None = None):
+    """MISA rows: router (if heads/r given), then top-k re-scored with the GPU's heads."""
+    rep = rep or Report()
+    k = wl.k if k is None else k
+    m = wl.m if m is None else m
+    Kf = oracle.widen_bf16(wl.K_bits)
+    Kbar_o = oracle.pool_keys(Kf, wl.key_offsets, wl.B)
+    if Kbar is not None:
+        err = np.abs(Kbar - Kbar_o)
+        if np.any(err > tol(Kbar_o)):
+            rep.fail(f"Kbar mismatch, max err {err.max():.3g}")
+    boff = oracle.block_offsets(wl.key_offsets, wl.B)
+    qs = wl.q_seq
+    for j, i in enumerate(rows):
+        s = int(qs[i])
+        t = int(wl.q_pos[i])
+        K_seq = Kf[int(wl.key_offsets[s]):int(wl.key_offsets[s + 1])]
+        q_t = oracle.widen_bf16(wl.q_bits[i])
+        w_t = wl.w[i].astype(np.float64)
+        r_o = oracle.router_scores(q_t, w_t, K_seq, Kbar_o[boff[s]:boff[s + 1]], t, wl.B)
+        use = None
+        if r is not None:
+            e = np.abs(r[j] - r_o)
+            rep.max_r_err = max(rep.max_r_err, float((e / tol(r_o)).max()))
+            if np.any(e > tol(r_o)):
+                rep.fail(f"row {i}: router score err {e.max():.3g}")
+        if heads is not None:
+            if not check_heads(rep, i, r_o, heads[j], m):
+                continue
+            use = np.asarray(heads[j], dtype=np.int64)
+        else:
+            use = oracle.route(r_o, m)
+        I = oracle.token_scores(q_t[use], w_t[use], K_seq[:t + 1])
+        check_topk(rep, i, I, idx[j], val[j], k)
+        rep.rows += 1
+    return rep
+
+
+def check_dense_rows(wl, rows, idx, val, k=None, rep: Report | None = None):
+    rep = rep or Report()
+    k = wl.k if k is None else k
+    Kf = oracle.widen_bf16(wl.K_bits)
+    qs = wl.q_seq
+    for j, i in enumerate(rows):
+        s = int(qs[i])
+        t = int(wl.q_pos[i])
+        K_seq = Kf[int(wl.key_offsets[s]):int(wl.key_offsets[s + 1])]
+        I = oracle.token_scores(oracle.widen_bf16(wl.q_bits[i]), wl.w[i].astype(np.float64),
+                                K_seq[:t + 1])
+        check_topk(rep, i, I, idx[j], val[j], k)
+        rep.rows += 1
+    return rep
+
+
+def check_rerank_rows(wl, rows, cand, idx, val, k=None, rep: Report | None = None):
+    """Re-rank of the GPU's own candidate rows against the oracle re-rank."""
+    rep = rep or Report()
+    k = wl.k if k is None else k
+    Kf = oracle.widen_bf16(wl.K_bits)
+    qs = wl.q_seq
+    for j, i in enumerate(rows):
+        s = int(qs[i])
+        K_seq = Kf[int(wl.key_offsets[s]):int(wl.key_offsets[s + 1])]
+        c = np.asarray(cand[j])
+        c = np.sort(c[c >= 0])
+        I_c = oracle.token_scores(oracle.widen_bf16(wl.q_bits[i]), wl.w[i].astype(np.float64),
+                                  K_seq[c])
+        check_topk(rep, i, I_c, idx[j], val[j], k, tokens=c)
+        rep.rows += 1
+    return rep

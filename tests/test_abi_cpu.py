@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every declared symbol; host-side
+argument checks answer without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def misa():
+    from long_context_sparse_misa_b200 import build
+    build.build()
+    import long_context_sparse_misa_b200 as m
+    return m
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "misa.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\*?\s+\*?(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points(misa):
+    names = declared_functions()
+    assert set(names) == set(misa.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(misa):
+    lib = ctypes.CDLL(misa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def _problem(misa, **kw):
+    d = dict(num_seqs=1, num_queries=4, num_heads=64, head_dim=128, block=64, max_seq_len=1000,
+             total_keys=1000, total_blocks=16, key_offsets=8, block_offsets=8, query_offsets=8,
+             q_pos=8)
+    d.update(kw)
+    return misa._Problem(**d)
+
+
+def test_workspace_size_and_validation(misa):
+    p = _problem(misa)
+    n = misa.lib.misa_workspace_size(ctypes.byref(p), 8, 2048, 0)
+    assert n >= 4 * 1000 * 4
+    assert misa.lib.misa_workspace_size(ctypes.byref(p), 65, 2048, 0) == 0      # m > H
+    bad = _problem(misa, head_dim=64)
+    assert misa.lib.misa_workspace_size(ctypes.byref(bad), 8, 10, 0) == 0
+    assert b"head_dim" in misa.lib.misa_last_error_string()
+    hier = misa.lib.misa_workspace_size(ctypes.byref(p), 8, 2048, 8192)
+    assert hier >= 4 * 8192 * 4
+
+
+def test_host_argument_errors_without_gpu(misa):
+    p = _problem(misa)
+    rp = ctypes.byref(p)
+    lib = misa.lib
+    # NULL pointers are rejected before any CUDA call
+    assert lib.misa_route(rp, None, None, None, None, 8, None, None, None, None, None, 0, None) == 1
+    assert lib.misa_score_topk(rp, None, None, 8, None, 16, None, None, None, 0, None, 0, None) == 1
+    # m not a power of two -> UNSUPPORTED; k out of range -> INVALID_ARG
+    assert lib.misa_score_topk(rp, 16, 16, 6, 16, 16, 16, 16, None, 0, 16, 1 << 20, None) == 2
+    assert lib.misa_score_topk(rp, 16, 16, 8, 16, 0, 16, 16, None, 0, 16, 1 << 20, None) == 1
+    # misaligned bf16 pointer
+    assert lib.misa_score_topk(rp, 18, 16, 8, 16, 16, 16, 16, None, 0, 16, 1 << 20, None) == 1
+    assert b"aligned" in lib.misa_last_error_string()
+    # hierarchical: k_cand < k
+    assert lib.misa_hier_rerank(rp, 16, 16, 16, 16, 10, 20, 16, 16, 16, 1 << 20, None) == 1
+    # dense needs H a power of two
+    p48 = _problem(misa, num_heads=48)
+    assert lib.dsa_index_dense(ctypes.byref(p48), 16, 16, 16, 8, 16, 16, None, 0, 16, 1 << 20,
+                               None) == 2
+    # workspace too small
+    assert lib.misa_route(rp, 16, 16, 16, 16, 8, 16, 16, 16, None, 16, 8, None) == 3
+    assert lib.misa_selftest_timeout(0, None) == 1
+    assert lib.misa_block_offsets(None, 1, 64, None, None) == 1
