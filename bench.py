@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--max-queries", type=int, default=0,
+                    help="keep only the last N queries (small captures for ncu)")
     return ap.parse_args()
 
 
@@ -267,6 +269,8 @@ def run_ours(args):
     world, rank, local = dist_init()
     cfg = args.config
     wl = make_config(cfg, seed=1000 + cfg + 100 * rank)
+    if args.max_queries and args.max_queries < wl.T:
+        wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
     hier = bool(wl.k_cand)
     dev = torch.device("cuda", torch.cuda.current_device())
     prob = misa.Problem.from_workload(wl, device=dev)

@@ -54,17 +54,20 @@ __global__ void block_offsets_kernel(const int64_t* __restrict__ ko, int S, int 
 }
 
 // One CTA: split every sequence's queries (restricted to [q_lo, q_hi)) into
-// groups of at most G and record {seq, q_begin, q_end, max_pos}.  Positions
-// outside their sequence are flagged.
+// groups of at most G and record {seq, q_begin, q_end, max_pos}.  A scan over
+// sequences gives each sequence its first group index; then every warp takes
+// groups round-robin and reduces the positions of its group's queries.
+// Positions outside their sequence are flagged and left out of max_pos.
 __global__ void plan_groups_kernel(const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
                                    const int32_t* __restrict__ q_pos, int S, int q_lo, int q_hi,
                                    int G, int4* __restrict__ groups, int* __restrict__ count,
                                    uint32_t* status) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
+  __shared__ int s_first[1024], s_ng[1024], s_b[1024], s_e[1024];
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int base = 0; base < S; base += blockDim.x) {
     const int s = base + threadIdx.x;
     int b = 0, e = 0, ng = 0;
@@ -82,7 +85,7 @@ __global__ void plan_groups_kernel(const int64_t* __restrict__ ko, const int32_t
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-      int ws = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+      int ws = lane < nwarps ? warp_sums[lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, ws, o);
@@ -92,17 +95,27 @@ __global__ void plan_groups_kernel(const int64_t* __restrict__ ko, const int32_t
     }
     __syncthreads();
     const int first = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - ng;
-    if (s < S) {
-      const int64_t L = ko[s + 1] - ko[s];
-      for (int g = 0; g < ng; ++g) {
-        const int qb = b + g * G, qe = min(qb + G, e);
+    s_first[threadIdx.x] = first;
+    s_ng[threadIdx.x] = ng;
+    s_b[threadIdx.x] = b;
+    s_e[threadIdx.x] = e;
+    __syncthreads();
+    const int nseq = min((int)blockDim.x, S - base);
+    for (int j = 0; j < nseq; ++j) {
+      const int ngj = s_ng[j];
+      if (ngj == 0) continue;
+      const int sj = base + j, bj = s_b[j], ej = s_e[j], fj = s_first[j];
+      const int64_t L = ko[sj + 1] - ko[sj];
+      for (int g = warp; g < ngj; g += nwarps) {
+        const int qb = bj + g * G, qe = min(qb + G, ej);
         int mp = -1;
-        for (int t = qb; t < qe; ++t) {
+        for (int t = qb + lane; t < qe; t += 32) {
           const int pos = q_pos[t];
           if (pos < 0 || pos >= L) set_status(status, MISA_STATUS_BAD_INPUT);
           else mp = max(mp, pos);
         }
-        groups[first + g] = make_int4(s, qb, qe, mp);
+        mp = __reduce_max_sync(0xffffffffu, mp);
+        if (lane == 0) groups[fj + g] = make_int4(sj, qb, qe, mp);
       }
     }
     __syncthreads();
