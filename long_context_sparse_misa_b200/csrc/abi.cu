@@ -213,11 +213,53 @@ int chunk_queries(const misa_problem_t* p, int64_t ld, size_t ws_bytes) {
   return 0;
 }
 
+int num_sms() {
+  int dev = 0, n = kSms;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : kSms;
+}
+
+// Streaming (fused top-k) scorer: used when every query scores its whole
+// prefix in groups that fill the GPU, no score rows are requested, and m fits.
+struct StreamPlan {
+  bool use = false;
+  int G = 0, grid = 0, max_groups = 0;
+  int64_t cap = 0;
+  size_t bytes = 0;
+};
+
+StreamPlan stream_plan(const misa_problem_t* p, int m, int k, bool want_rows) {
+  StreamPlan sp;
+  if (want_rows || (m != 8 && m != 16 && m != 32 && m != 64) || k > 16384) return sp;
+  sp.G = stream_group_size(m);
+  const int T = p->num_queries;
+  sp.max_groups = (T + sp.G - 1) / sp.G + p->num_seqs;
+  const int sms = num_sms();
+  if ((T / sp.G) < 2 * sms) return sp;  // too few groups: split the keys instead
+  sp.grid = sms < sp.max_groups ? sms : sp.max_groups;
+  sp.cap = stream_subcap(p->max_seq_len);
+  sp.bytes = groups_bytes(T, p->num_seqs) + align_up(stream_cand_bytes(sp.grid, sp.cap));
+  sp.use = true;
+  return sp;
+}
+
 int score_topk_impl(const misa_problem_t* p, const uint16_t* qsel, const float* wsel, int m,
                     const uint16_t* K, int k, int32_t* idx, float* val, float* scores_dbg,
                     int64_t scores_ld, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int T = p->num_queries;
   if (T == 0) return MISA_OK;
+  const StreamPlan sp = stream_plan(p, m, k, scores_dbg != nullptr);
+  if (sp.use && ws_bytes >= sp.bytes) {
+    Carve c = carve(ws, T, p->num_seqs);
+    int rc = launch_plan_groups(*p, 0, T, sp.G, c.groups, c.count, st);
+    if (rc) return rc;
+    StreamArgs a;
+    a.p = p; a.qsel = qsel; a.wsel = wsel; a.m = m; a.K = K; a.groups = c.groups;
+    a.group_count = c.count; a.max_groups = sp.max_groups; a.grid = sp.grid; a.k = k;
+    a.cand = reinterpret_cast<uint2*>(c.buf); a.subcap = sp.cap; a.idx = idx; a.val = val;
+    return launch_score_stream(a, st);
+  }
   const int64_t ld = scores_dbg ? scores_ld : row_ld(p);
   int chunk = T;
   if (!scores_dbg) {
@@ -298,6 +340,12 @@ size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_
   if (k_cand > 0) {
     const size_t hr = groups_bytes(T, S) + align_up((size_t)T * k_cand * 4);
     if (hr > need) need = hr;
+  }
+  // streaming scorer for the routed heads (m) and for the dense indexer (H)
+  const int ks = k_cand > k ? k_cand : k;
+  for (int mm : {m, p->num_heads}) {
+    const StreamPlan sp = stream_plan(p, mm, ks, false);
+    if (sp.use && sp.bytes > need) need = sp.bytes;
   }
   return need;
 }

@@ -82,6 +82,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// All 32 lanes wait together; the outcome is warp-uniform (so .sync.aligned
+// tcgen05 instructions that follow are executed by the whole warp or by none).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* abort,
+                                          uint32_t* status, long long limit = kWaitCycles) {
+  const int lane = threadIdx.x & 31;
+  long long t0 = 0;
+  if (lane == 0) t0 = clock64();
+  while (true) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    int give_up = 0;
+    if (lane == 0) {
+      if (*reinterpret_cast<volatile int*>(abort)) {
+        give_up = 1;
+      } else if (clock64() - t0 > limit) {
+        *reinterpret_cast<volatile int*>(abort) = 1;
+        set_status(status, MISA_STATUS_TIMEOUT);
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -196,6 +220,55 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Ties 32 registers filled by tcgen05.ld to a point after tcgen05.wait::ld:
+// the empty volatile asm is ordered after the wait, and every later use reads
+// its outputs, so the compiler cannot hoist a use above the wait.
+__device__ __forceinline__ void reg_fence32(float (&v)[32]) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                 "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]),
+                 "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+                 "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]),
+                 "+f"(v[30]), "+f"(v[31]));
+}
+
+// a0 += w0 * r0 and a1 += w1 * r1 as one packed fp32 FMA (sm_100 f32x2).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float r0,
+                                      float r1) {
+  uint64_t a, w, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(w) : "f"(w0), "f"(w1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(r0), "f"(r1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(w), "l"(r));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
+}
+
+// Head-weighted ReLU sum of one query's MH accumulator columns, the one
+// summation order every scoring kernel uses (so all paths agree bit for bit):
+// even heads into a0, odd heads into a1 (one packed FMA per pair), then
+// a0 + a1.  `col(j)` gives the accumulator value of head j, `wq` the head
+// weights.
+template <int MH, typename ColFn>
+__device__ __forceinline__ float relu_wsum(ColFn col, const float* wq) {
+  float a0 = 0.f, a1 = 0.f;
+  if constexpr (MH == 1) {
+    a0 = fmaf(wq[0], fmaxf(col(0), 0.f), a0);
+  } else {
+#pragma unroll
+    for (int j = 0; j < MH; j += 2) {
+      const float2 wj = *reinterpret_cast<const float2*>(wq + j);
+      ffma2(a0, a1, wj.x, wj.y, fmaxf(col(j), 0.f), fmaxf(col(j + 1), 0.f));
+    }
+  }
+  return a0 + a1;
+}
+
+// Inverse of order_key (for bin edges).
+__device__ __forceinline__ float key_to_float(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
 // ---------------------------------------------------------------- ordering keys

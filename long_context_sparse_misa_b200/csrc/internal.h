@@ -76,6 +76,28 @@ struct ScoreArgs {
   int max_tiles;          // host bound on key tiles per group
 };
 int launch_score(const ScoreArgs& a, cudaStream_t st);
+
+// ---- score_stream.cu: scoring with the top-k fused (every query's full prefix).
+struct StreamArgs {
+  const misa_problem_t* p;
+  const uint16_t* qsel;   // [T * m, 128] bf16
+  const float* wsel;      // [T, m]
+  int m;                  // 8, 16, 32 or 64
+  const uint16_t* K;
+  const int4* groups;     // G = stream_group_size(m) queries per group
+  const int* group_count;
+  int max_groups;
+  int grid;               // persistent CTAs (<= number of SMs)
+  int k;
+  uint2* cand;            // [grid * 32 queries * 4 quarters, subcap] candidate buffers
+  int64_t subcap;         // stream_subcap(max_seq_len)
+  int32_t* idx;
+  float* val;
+};
+int launch_score_stream(const StreamArgs& a, cudaStream_t st);
+int stream_group_size(int m);
+size_t stream_cand_bytes(int grid, int64_t subcap);
+int64_t stream_subcap(int max_seq_len);
 int score_group_size(int m);
 
 // ---- topk.cu

@@ -74,29 +74,6 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-// All 32 lanes wait together; the outcome is warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* abort,
-                                          uint32_t* status) {
-  const int lane = threadIdx.x & 31;
-  long long t0 = 0;
-  if (lane == 0) t0 = clock64();
-  while (true) {
-    const bool done = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, done)) return true;
-    int give_up = 0;
-    if (lane == 0) {
-      if (*reinterpret_cast<volatile int*>(abort)) {
-        give_up = 1;
-      } else if (clock64() - t0 > kWaitCycles) {
-        *reinterpret_cast<volatile int*>(abort) = 1;
-        set_status(status, MISA_STATUS_TIMEOUT);
-        give_up = 1;
-      }
-    }
-    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
-  }
-}
-
 template <int MH, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -276,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int lrow = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int nchunks = NP / 32;
+    const int nwin = (NP + 63) / 64;
     for (int i = 0; i < nt; ++i) {
       const int buf = i & 1;
       if (!warp_wait(&s.tfull[buf], (i >> 1) & 1, s.abort, status)) break;
@@ -290,42 +267,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (key >= 0 && !key_ok) set_status(status, MISA_STATUS_BAD_INPUT);
       }
       const uint32_t taddr = lane_addr + buf * kMaxN;
-      float acc = 0.f;
-      for (int c = 0; c < nchunks; ++c) {
-        float v[32];
-        tmem_ld32(taddr + c * 32, v);
+      for (int c = 0; c < nwin; ++c) {
+        // 64-column window (the buffer has kMaxN columns, so reading past NP is harmless)
+        float v[2][32];
+        tmem_ld32(taddr + c * 64, v[0]);
+        tmem_ld32(taddr + c * 64 + 32, v[1]);
         tmem_wait_ld();
-        if constexpr (MH <= 32) {
-          constexpr int QPC = 32 / MH;
+        reg_fence32(v[0]);
+        reg_fence32(v[1]);
+        constexpr int QPW = 64 / MH;  // queries per 64-column window
 #pragma unroll
-          for (int qq = 0; qq < QPC; ++qq) {
-            const int qi = c * QPC + qq;
-            if (qi >= nq) break;
-            const float* wq = s.w + qi * MH;
-            float sc = 0.f;
-#pragma unroll
-            for (int j = 0; j < MH; ++j) sc = fmaf(wq[j], fmaxf(v[qq * MH + j], 0.f), sc);
-            if (GATHER) {
-              if (slot < k_cand && s.row[0] >= 0)
-                I[(int64_t)s.row[0] * ld + slot] = key_ok ? sc : -INFINITY;
-            } else if (key <= s.pos[qi]) {
-              I[(int64_t)s.row[qi] * ld + key] = sc;
-            }
-          }
-        } else {
-          constexpr int CPQ = MH / 32;
-          const int qi = c / CPQ;
-          const float* wq = s.w + c * 32;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
-          if ((c % CPQ) == CPQ - 1) {
-            if (GATHER) {
-              if (slot < k_cand && s.row[0] >= 0)
-                I[(int64_t)s.row[0] * ld + slot] = key_ok ? acc : -INFINITY;
-            } else if (qi < nq && key <= s.pos[qi]) {
-              I[(int64_t)s.row[qi] * ld + key] = acc;
-            }
-            acc = 0.f;
+        for (int qq = 0; qq < QPW; ++qq) {
+          const int qi = c * QPW + qq;
+          if (qi >= nq) break;
+          const float sc = relu_wsum<MH>(
+              [&](int j) {
+                const int col = qq * MH + j;
+                return v[col >> 5][col & 31];
+              },
+              s.w + qi * MH);
+          if (GATHER) {
+            if (slot < k_cand && s.row[0] >= 0)
+              I[(int64_t)s.row[0] * ld + slot] = key_ok ? sc : -INFINITY;
+          } else if (key <= s.pos[qi]) {
+            I[(int64_t)s.row[qi] * ld + key] = sc;
           }
         }
       }

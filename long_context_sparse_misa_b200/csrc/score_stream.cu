@@ -1,0 +1,613 @@
+// Routed token scoring with the per-query top-k fused into the epilogue
+// (prefill: every query scores its whole causal prefix).
+//
+// "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference",
+// gist.science summary, "Methodologie: MISA" (Sparse Token Scoring: only the
+// routed heads score the prefix; the top-k tokens come from those scores).
+// The same kernel with m = H is the dense DSA indexer (abstract).
+//
+// Why fused: at 128K prefill the score matrix is 8.6e9 fp32 values (34 GB);
+// writing and re-reading it costs more than the tensor-core work.  Here no
+// score leaves the SM unless it can still be in its query's top-k.
+//
+// CTA (persistent, one per SM): query groups of G = 256/m queries taken
+// longest-prefix first, round-robin over CTAs.  Per group: the group's
+// (query, head) rows stay in shared memory (B operand, N = 256); 128-key
+// tiles of K stream through a 4-stage TMA ring (A operand); tcgen05.mma
+// accumulates 128 keys x 256 columns in TMEM, two buffers.
+//
+// Epilogue (8 warps: TMEM lane quarter = warp % 4, column half = which of
+// the two warps of that quarter), per tile: two tcgen05.ld of 32 columns
+// before each wait, the TMEM buffer released after the second pair, then per
+// key and query I = sum_j w_j ReLU(acc_j), the causal mask, and the
+// streaming selection:
+//   * tau_q, a safe lower bound on query q's k-th best score: a key is
+//     appended to q's candidate buffer only if I >= tau_q.  Each (query,
+//     lane quarter) has a private sub-buffer with one slot per key the
+//     quarter can see, so nothing can overflow and the slot counter lives in
+//     a register (no returning atomics on the hot path).
+//   * a 128-bin histogram per query (1/8-octave bins of the order-preserving
+//     score key, anchored 14 octaves below the first tile's maximum) counts
+//     the appended scores; every other tile the owner warp raises tau_q to the
+//     lower edge of the bin where the count from the top reaches k.  At least
+//     k appended scores are >= that edge, so a later key scoring below it
+//     cannot be in the top-k whatever its index; equal scores are kept, so
+//     ties resolved by token index stay exact.  Reads of the histogram race
+//     with other warps' appends only towards a lower (still safe) tau.
+//   * at the end of the group the owner warp selects exactly: entries above
+//     the histogram's threshold bin are taken, the threshold bin is resolved
+//     by a warp-level radix select over (score, lower index first).
+#include "common.cuh"
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiWarps = 8;
+constexpr int kStages = 4;
+constexpr int kStageBytes = kTileKeys * kD * 2;  // 32 KB
+constexpr int kHalfBytes = kStageBytes / 2;
+constexpr int kN = 256;                          // MMA N = group columns
+constexpr int kQHalfBytes = kN * 128;            // 32 KB per 64-dim half
+constexpr int kQBytes = 2 * kQHalfBytes;
+constexpr int kTmemCols = 2 * kN;
+constexpr int kMaxG = 32;                        // queries per group (m >= 8)
+constexpr int kBins = 128;
+constexpr int kBinShift = 20;                    // 12-bit score key prefix: 1/8 octave
+constexpr int kHeadroom = 112;                   // bins below the first tile's maximum
+constexpr int kSelBins = 256;
+
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
+                           kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ + kMaxG * 4 * 4 /*wc*/ +
+                           kMaxG * kBins * 4 /*hist*/ + kEpiWarps * kSelBins * 4 /*select*/ +
+                           32 * 8 /*barriers*/ + 16;
+
+struct Smem {
+  uint8_t* q;
+  uint8_t* k;
+  float* w;
+  int* pos;
+  int* row;
+  float* tau;
+  uint32_t* maxkey;
+  int* base;  // histogram anchor per query
+  int* wc;    // [kMaxG][4] sub-buffer counts
+  uint32_t* hist;
+  uint32_t* sel;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* qfull;
+  uint64_t* qempty;
+  uint64_t* ebar;
+  uint64_t* drain;
+  uint32_t* tmem_slot;
+  int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* p =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.q = p;
+  s.k = p + kQBytes;
+  s.w = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
+  s.pos = reinterpret_cast<int*>(s.w + kN);
+  s.row = s.pos + kMaxG;
+  s.tau = reinterpret_cast<float*>(s.row + kMaxG);
+  s.maxkey = reinterpret_cast<uint32_t*>(s.tau + kMaxG);
+  s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
+  s.wc = s.base + kMaxG;
+  s.hist = reinterpret_cast<uint32_t*>(s.wc + kMaxG * 4);
+  s.sel = s.hist + kMaxG * kBins;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.sel + kEpiWarps * kSelBins);
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = s.tfull + 2;
+  s.qfull = s.tempty + 2;
+  s.qempty = s.qfull + 1;
+  s.ebar = s.qempty + 1;
+  s.drain = s.ebar + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
+  return s;
+}
+
+// Histogram anchor of a query: 14 octaves below its first tile's maximum.
+__device__ __forceinline__ int hist_base(uint32_t maxkey) {
+  const int b = static_cast<int>(maxkey >> kBinShift) - kHeadroom;
+  return b < 0 ? 0 : b;
+}
+
+__device__ __forceinline__ int score_bin(uint32_t key, int base) {
+  const int b = static_cast<int>(key >> kBinShift) - base;
+  return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
+}
+
+// Barrier over the 8 epilogue warps (bounded; warp-uniform result).
+__device__ __forceinline__ bool ep_barrier(Smem& s, uint32_t& phase, uint32_t* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(s.ebar);
+  const bool ok = warp_wait(s.ebar, phase, s.abort, status);
+  phase ^= 1u;
+  return ok;
+}
+
+// 64-bit selection key: score order first, then the lower token index.
+__device__ __forceinline__ uint64_t sel_key(uint2 e) {
+  return (static_cast<uint64_t>(order_key(__uint_as_float(e.x))) << 32) |
+         static_cast<uint64_t>(0xFFFFFFFFu - e.y);
+}
+
+// Bin (of `nb` descending-ordered counts, `per` per lane) where the count
+// from the top reaches `need`; returns bin, count above it and its count.
+template <int PER>
+__device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint32_t need,
+                                              int& bin, uint32_t& above_out, uint32_t& cnt_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t c[PER], loc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    c[i] = hist[nb - 1 - (lane * PER + i)];
+    loc += c[i];
+  }
+  uint32_t inc = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  uint32_t above = inc - loc;
+  int mb = -1;
+  uint32_t ma = 0, mc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    if (above < need && above + c[i] >= need) {
+      mb = nb - 1 - (lane * PER + i);
+      ma = above;
+      mc = c[i];
+    }
+    above += c[i];
+  }
+  const uint32_t who = __ballot_sync(0xffffffffu, mb >= 0);
+  if (!who) {
+    bin = -1;
+    above_out = cnt_out = 0;
+    return;
+  }
+  const int src = __ffs(who) - 1;
+  bin = __shfl_sync(0xffffffffu, mb, src);
+  above_out = __shfl_sync(0xffffffffu, ma, src);
+  cnt_out = __shfl_sync(0xffffffffu, mc, src);
+}
+
+// Exact top-k of one query's four candidate sub-buffers (region[r*subcap ..],
+// counts nr[r]), by one warp.  Threshold-bin entries are compacted in order
+// to the front of the region, which never overtakes the entries still to be
+// read.
+__device__ void final_select(uint2* region, int64_t subcap, const int* nr, const uint32_t* hist,
+                             int base, int k, int32_t* idx, float* val, uint32_t* selh) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int n = nr[0] + nr[1] + nr[2] + nr[3];
+  int out = 0;
+  if (n <= k) {
+    for (int r = 0; r < 4; ++r) {
+      const uint2* sb = region + r * subcap;
+      for (int j = lane; j < nr[r]; j += 32) {
+        const uint2 e = sb[j];
+        idx[out + j] = static_cast<int32_t>(e.y);
+        val[out + j] = __uint_as_float(e.x) + 0.0f;
+      }
+      out += nr[r];
+    }
+  } else {
+    int bstar;
+    uint32_t A, Z;
+    find_crossing<4>(hist, kBins, (uint32_t)k, bstar, A, Z);
+    uint32_t need = (uint32_t)k - A;
+    // Pass 1: entries above the threshold bin go out; threshold-bin entries
+    // are compacted to the front of the region.  Each lane issues kU loads
+    // before using any of them (the buffer is mostly beyond L2).
+    constexpr int kU = 8;
+    int zpos = 0;
+    for (int r = 0; r < 4; ++r) {
+      const uint2* sb = region + r * subcap;
+      const int nrr = nr[r];
+      for (int j0 = 0; j0 < nrr; j0 += 32 * kU) {
+        uint2 ev[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int j = j0 + u * 32 + lane;
+          ev[u] = j < nrr ? __ldcs(sb + j) : make_uint2(0u, 0u);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int j = j0 + u * 32 + lane;
+          const uint2 e = ev[u];
+          const int b = j < nrr ? score_bin(order_key(__uint_as_float(e.x)), base) : -1;
+          const uint32_t up = __ballot_sync(0xffffffffu, b > bstar);
+          if (b > bstar) {
+            const int o = out + __popc(up & lt);
+            idx[o] = static_cast<int32_t>(e.y);
+            val[o] = __uint_as_float(e.x) + 0.0f;
+          }
+          out += __popc(up);
+          const uint32_t zb = __ballot_sync(0xffffffffu, b == bstar);
+          if (b == bstar) region[zpos + __popc(zb & lt)] = e;
+          zpos += __popc(zb);
+        }
+        __syncwarp();
+      }
+    }
+    __syncwarp();
+    // Pass 2: choose `need` of the Z threshold-bin entries by exact key.
+    int shift = 64;
+    uint64_t prefix = 0;
+    if (need < Z) {
+      for (int p = 0; p < 8; ++p) {
+        const int sh = 56 - 8 * p;
+        for (int i = lane; i < kSelBins; i += 32) selh[i] = 0;
+        __syncwarp();
+        for (int j = lane; j < (int)Z; j += 32) {
+          const uint64_t key = sel_key(region[j]);
+          if (p == 0 || (key >> (sh + 8)) == prefix) atomicAdd(&selh[(key >> sh) & 255u], 1u);
+        }
+        __syncwarp();
+        int bin;
+        uint32_t ab, cnt;
+        find_crossing<8>(selh, kSelBins, need, bin, ab, cnt);
+        need -= ab;
+        prefix = (prefix << 8) | static_cast<uint64_t>(bin);
+        shift = sh;
+        __syncwarp();
+        if (cnt == need) break;
+      }
+    }
+    for (int j0 = 0; j0 < (int)Z; j0 += 32) {
+      const int j = j0 + lane;
+      bool take = false;
+      uint2 e = make_uint2(0u, 0u);
+      if (j < (int)Z) {
+        e = region[j];
+        take = shift == 64 || (sel_key(e) >> shift) >= prefix;
+      }
+      const uint32_t tb = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const int o = out + __popc(tb & lt);
+        if (o < k) {
+          idx[o] = static_cast<int32_t>(e.y);
+          val[o] = __uint_as_float(e.x) + 0.0f;
+        }
+      }
+      out += __popc(tb);
+    }
+  }
+  for (int j = out + lane; j < k; j += 32) {
+    idx[j] = -1;
+    val[j] = -INFINITY;
+  }
+}
+
+template <int MH>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_stream_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap qmap, const float* __restrict__ wsel,
+                        const int32_t* __restrict__ q_pos, const int64_t* __restrict__ ko,
+                        const int4* __restrict__ groups, const int* __restrict__ group_count,
+                        int k, uint2* __restrict__ cand, int64_t subcap,
+                        int32_t* __restrict__ idx_out, float* __restrict__ val_out,
+                        uint32_t* status) {
+  constexpr int G = kN / MH;          // queries per group
+  constexpr int QH = G / 2;           // queries per column half
+  constexpr int QPW = QH / 2;         // queries per 64-column window
+  static_assert(MH >= 8 && MH <= 64 && G <= kMaxG && QPW >= 1, "unsupported head count");
+  extern __shared__ uint8_t smem_raw[];
+
+  const int count = *group_count;
+  if ((int)blockIdx.x >= count) return;
+
+  Smem s = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], kEpiWarps);
+    }
+    mbar_init(s.qfull, 1);
+    mbar_init(s.qempty, 1);
+    mbar_init(s.ebar, kEpiWarps);
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&qmap);
+      int it = 0, gl = 0;
+      bool ok = true;
+      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+        const int4 grp = groups[count - 1 - gs];
+        if (grp.w < 0) continue;  // no valid query in the group
+        const int64_t key_base = ko[grp.x];
+        const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+        if (!(ok = mbar_wait(s.qempty, (gl & 1) ^ 1, s.abort, status))) break;
+        mbar_arrive_expect_tx(s.qfull, kQBytes);
+        for (int h = 0; h < 2; ++h)
+          for (int r0 = 0; r0 < kN; r0 += 32)
+            tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
+                        grp.y * MH + r0);
+        ++gl;
+        for (int i = 0; i < ntiles; ++i, ++it) {
+          const int st = it % kStages;
+          if (!(ok = mbar_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, s.abort, status))) break;
+          mbar_arrive_expect_tx(&s.full[st], kStageBytes);
+          const int32_t krow = (int32_t)(key_base + (int64_t)i * kTileKeys);
+          uint8_t* dst = s.k + st * kStageBytes;
+          tma_load_2d(&kmap, &s.full[st], dst, 0, krow);
+          tma_load_2d(&kmap, &s.full[st], dst + kHalfBytes, 64, krow);
+        }
+      }
+      // Drain this CTA's copies before it exits.
+      for (int i = max(0, it - kStages); i < it; ++i)
+        mbar_wait(&s.full[i % kStages], (i / kStages) & 1, s.abort, status, kDrainCycles, true);
+      if (gl > 0) mbar_wait(s.qfull, (gl - 1) & 1, s.abort, status, kDrainCycles, true);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileKeys, kN);
+      const uint32_t q_addr = smem_u32(s.q);
+      int it = 0, tb = 0, gl = 0;
+      bool ok = true;
+      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+        const int4 grp = groups[count - 1 - gs];
+        if (grp.w < 0) continue;
+        const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+        if (!(ok = mbar_wait(s.qfull, gl & 1, s.abort, status))) break;
+        tc_fence_after();
+        for (int i = 0; i < ntiles; ++i, ++it, ++tb) {
+          const int st = it % kStages, buf = tb & 1;
+          if (!(ok = mbar_wait(&s.full[st], (it / kStages) & 1, s.abort, status))) break;
+          if (!(ok = mbar_wait(&s.tempty[buf], ((tb >> 1) & 1) ^ 1, s.abort, status))) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(s.k + st * kStageBytes);
+          const uint32_t d = tmem_base + buf * kN;
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t a = sw128_kmajor_desc(k_addr + (kk >> 2) * kHalfBytes + off);
+            const uint64_t b = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes + off);
+            umma_bf16(d, a, b, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s.empty[st]);
+          umma_commit(&s.tfull[buf]);
+        }
+        umma_commit(s.qempty);  // the group's rows may be replaced once these MMAs are done
+        ++gl;
+      }
+      umma_commit(s.drain);
+      mbar_wait(s.drain, 0, s.abort, status, kDrainCycles, true);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;                  // 0..7
+    const int quarter = warp & 3;            // TMEM lane quarter of this warp
+    const int half = e >> 2;                 // column half: queries half*QH .. half*QH+QH-1
+    const int lrow = quarter * 32 + lane;    // key row of the tile
+    const int et = threadIdx.x - 64;         // 0..255
+    const uint32_t lt = (1u << lane) - 1u;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t ephase = 0;
+    int tb = 0;
+    bool ok = true;
+    for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+      const int4 grp = groups[count - 1 - gs];
+      if (grp.w < 0) continue;
+      const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
+      const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+      const int64_t L = ko[seq + 1] - ko[seq];
+      // Group state: column weights, query limits, selection state.
+      {
+        const int qi = et / MH;
+        s.w[et] = qi < nq ? wsel[(int64_t)(qb + qi) * MH + (et - qi * MH)] : 0.f;
+      }
+      if (et < G) {
+        int p = -1;
+        if (et < nq) {
+          p = q_pos[qb + et];
+          if (p < 0 || p >= L) p = -1;
+        }
+        s.pos[et] = p;
+        s.row[et] = qb + et;
+        s.tau[et] = -INFINITY;
+        s.maxkey[et] = 0u;
+      }
+      for (int i = et; i < G * kBins; i += 256) s.hist[i] = 0u;
+      // This warp's slot counters (one per query; only this warp touches
+      // them) and its sub-buffer of its first query; query stride 4 * subcap.
+      int* mycnt = s.wc + (half * QH) * 4 + quarter;
+      if (lane < QH) mycnt[lane * 4] = 0;
+      uint2* mysub = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 4 * subcap +
+                     (int64_t)quarter * subcap;
+      const int qstride = 4 * static_cast<int>(subcap);
+      if (!(ok = ep_barrier(s, ephase, status))) break;
+      float tauR[QH];  // this warp's copy of its queries' thresholds (refreshed every 4 tiles)
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) tauR[qq] = -INFINITY;
+
+      for (int i = 0; i < ntiles; ++i, ++tb) {
+        const int buf = tb & 1;
+        if (!(ok = warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status))) break;
+        tc_fence_after();
+        const uint32_t taddr = lane_addr + buf * kN + half * 128;
+        float sc[QH];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[2][32];
+          tmem_ld32(taddr + (2 * hh) * 32, v[0]);
+          tmem_ld32(taddr + (2 * hh + 1) * 32, v[1]);
+          tmem_wait_ld();
+          reg_fence32(v[0]);
+          reg_fence32(v[1]);
+          if (hh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[buf]);
+          }
+#pragma unroll
+          for (int q2 = 0; q2 < QPW; ++q2) {
+            sc[hh * QPW + q2] = relu_wsum<MH>(
+                [&](int j) {
+                  const int col = q2 * MH + j;
+                  return v[col >> 5][col & 31];
+                },
+                s.w + half * 128 + hh * 64 + q2 * MH);
+          }
+        }
+        const int key = i * kTileKeys + lrow;
+        if (i == 0) {
+          // Anchor every query's histogram at its first tile's maximum.
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) {
+            const int qi = half * QH + qq;
+            uint32_t kk = key <= s.pos[qi] ? order_key(sc[qq]) : 0u;
+            kk = __reduce_max_sync(0xffffffffu, kk);
+            if (lane == 0) atomicMax(&s.maxkey[qi], kk);
+          }
+          if (!(ok = ep_barrier(s, ephase, status))) break;
+          // every warp of a half writes the same anchors for its queries
+          if (lane < QH) s.base[half * QH + lane] = hist_base(s.maxkey[half * QH + lane]);
+          __syncwarp();
+        }
+        if ((i & 3) == 0) {
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
+        }
+        // Streaming selection: every ballot first, then the appends.
+        uint32_t bal[QH];
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq)
+          bal[qq] = __ballot_sync(0xffffffffu, key <= s.pos[half * QH + qq] && sc[qq] >= tauR[qq]);
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) {
+          if (bal[qq]) {
+            const int c0 = mycnt[qq * 4];
+            if ((bal[qq] >> lane) & 1u) {
+              const int qi = half * QH + qq;
+              mysub[qq * qstride + c0 + __popc(bal[qq] & lt)] =
+                  make_uint2(__float_as_uint(sc[qq]), static_cast<uint32_t>(key));
+              atomicAdd(&s.hist[qi * kBins + score_bin(order_key(sc[qq]), s.base[qi])], 1u);
+            }
+            __syncwarp();
+            if (lane == 0) mycnt[qq * 4] = c0 + __popc(bal[qq]);
+          }
+        }
+        // Owner warps raise tau for their queries (qi % 8 == e), every 4th tile.
+        if ((i & 3) == 3) {
+          for (int qi = e; qi < G; qi += kEpiWarps) {
+            int bstar;
+            uint32_t A, Z;
+            find_crossing<4>(s.hist + qi * kBins, kBins, (uint32_t)k, bstar, A, Z);
+            if (lane == 0 && bstar > 0) {
+              const float edge =
+                  key_to_float(static_cast<uint32_t>(s.base[qi] + bstar) << kBinShift);
+              if (edge > s.tau[qi]) s.tau[qi] = edge;
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      if (!(ok = ep_barrier(s, ephase, status))) break;
+      for (int qi = e; qi < nq; qi += kEpiWarps) {
+        const int t = s.row[qi];
+        if (s.pos[qi] < 0) {  // invalid position: padded row
+          for (int j = lane; j < k; j += 32) {
+            idx_out[(int64_t)t * k + j] = -1;
+            val_out[(int64_t)t * k + j] = -INFINITY;
+          }
+          continue;
+        }
+        uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 4 * subcap;
+        final_select(region, subcap, s.wc + qi * 4, s.hist + qi * kBins,
+                     s.base[qi], k, idx_out + (int64_t)t * k,
+                     val_out + (int64_t)t * k, s.sel + e * kSelBins);
+      }
+      if (!(ok = ep_barrier(s, ephase, status))) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int MH>
+int launch_one(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap,
+               cudaStream_t st) {
+  auto kern = score_stream_kernel<MH>;
+  int rc = set_smem_limit((const void*)kern, kSmemBytes);
+  if (rc) return rc;
+  ProfScope ps("score", st);
+  kern<<<a.grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.wsel, a.p->q_pos, a.p->key_offsets,
+                                            a.groups, a.group_count, a.k, a.cand, a.subcap,
+                                            a.idx, a.val, status_ptr());
+  return cuda_fail(cudaGetLastError(), "score_stream_kernel");
+}
+
+}  // namespace
+
+int stream_group_size(int m) { return kN / m; }
+
+int64_t stream_subcap(int max_seq_len) {
+  // keys one lane quarter can see: 32 per 128-key tile
+  return ((int64_t)max_seq_len + kTileKeys - 1) / kTileKeys * 32;
+}
+
+size_t stream_cand_bytes(int grid, int64_t subcap) {
+  return (size_t)grid * kMaxG * 4 * (size_t)subcap * sizeof(uint2);
+}
+
+int launch_score_stream(const StreamArgs& a, cudaStream_t st) {
+  if (a.max_groups <= 0) return MISA_OK;
+  CUtensorMap kmap, qmap;
+  int rc = make_kmajor_map(&kmap, a.K, a.p->total_keys, kTileKeys);
+  if (rc) return rc;
+  rc = make_kmajor_map(&qmap, a.qsel, (int64_t)a.p->num_queries * a.m, 32);
+  if (rc) return rc;
+  switch (a.m) {
+    case 8: return launch_one<8>(a, kmap, qmap, st);
+    case 16: return launch_one<16>(a, kmap, qmap, st);
+    case 32: return launch_one<32>(a, kmap, qmap, st);
+    case 64: return launch_one<64>(a, kmap, qmap, st);
+    default:
+      set_error("streaming scorer needs m in {8,16,32,64}, got %d", a.m);
+      return MISA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace misa

@@ -1,0 +1,151 @@
+"""The streaming scorer (top-k fused into the tcgen05 epilogue) vs the
+materialised-rows path and the CPU oracle, through the C ABI (B200 only).
+
+The streaming path is chosen by the library when there are enough query
+groups to fill the GPU (here: prefills of about 10K queries); passing a
+scores_dbg buffer forces the materialised path on the same inputs.  Both
+compute bit-identical scores, so their selections must be identical.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_sparse_misa_b200 as misa
+import oracle
+from misa_synth import f32_to_bf16_bits, make_workload
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(wl):
+    prob = misa.Problem.from_workload(wl)
+    return (prob, torch.from_numpy(wl.K_bits).cuda(), torch.from_numpy(wl.q_bits).cuda(),
+            torch.from_numpy(wl.w).cuda())
+
+
+def status_ok():
+    code, bits = misa.stream_status()
+    assert code == 0 and bits == 0, f"device status {code}/{bits}"
+
+
+def run_both(wl, dense=False):
+    """(stream idx, stream val, rows idx, rows val, heads) for one workload."""
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    L = int(wl.seq_lens.max())
+    dbg = torch.empty((wl.T, L), dtype=torch.float32, device="cuda")
+    misa.profile_enable(True)
+    if dense:
+        ix.dense(q, w, K)
+    else:
+        ix.misa(q, w, K)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    si, sv = ix.idx.clone(), ix.val.clone()
+    if dense:
+        ix.dense(q, w, K, scores_dbg=dbg)
+    else:
+        misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, K, wl.k, ix.idx, ix.val, ix.ws, dbg)
+    status_ok()
+    assert "topk" not in prof, "streaming path was not taken"
+    return si, sv, ix.idx, ix.val, ix.heads
+
+
+def same_sets(si, sv, ri, rv):
+    a, b = torch.sort(si, dim=1), torch.sort(ri, dim=1)
+    assert torch.equal(a.values, b.values), "selections differ"
+    va = torch.gather(sv, 1, a.indices)
+    vb = torch.gather(rv, 1, b.indices)
+    assert torch.equal(va, vb), "values differ"
+
+
+def invariants(wl, idx):
+    n = torch.from_numpy(wl.q_pos.astype(np.int64) + 1).cuda()
+    valid = idx >= 0
+    assert torch.equal(valid.sum(1), torch.clamp(n, max=wl.k))
+    assert bool((idx <= (n - 1)[:, None]).all())
+    srt = torch.sort(idx, dim=1).values
+    assert not bool(((srt[:, 1:] == srt[:, :-1]) & (srt[:, 1:] >= 0)).any())
+
+
+def sample_rows(wl, n=80):
+    rng = np.random.default_rng(1)
+    rows = set(rng.choice(wl.T, n, replace=False).tolist())
+    rows |= {0, 1, wl.k - 1, wl.k, wl.k + 1, wl.T - 1}
+    return sorted(r for r in rows if r < wl.T)
+
+
+@pytest.mark.parametrize("H,m,B,k", [(32, 8, 128, 256), (64, 8, 64, 2048), (32, 16, 128, 100),
+                                     (64, 8, 64, 1)])
+def test_stream_matches_rows_and_oracle(H, m, B, k):
+    wl = make_workload(seq_lens=[10000], queries="all", H=H, B=B, m=m, k=k, seed=H + k)
+    si, sv, ri, rv, heads = run_both(wl)
+    same_sets(si, sv, ri, rv)
+    invariants(wl, si)
+    rows = sample_rows(wl)
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_misa_rows(wl, rows, si[sel].cpu().numpy(), sv[sel].cpu().numpy(),
+                           heads=heads[sel].cpu().numpy(), k=k, m=m).assert_ok()
+
+
+def test_stream_dense_multi_sequence():
+    wl = make_workload(seq_lens=[5000, 3000, 2700], queries="all", H=32, B=128, m=8, k=512,
+                       seed=9)
+    si, sv, ri, rv, _ = run_both(wl, dense=True)
+    same_sets(si, sv, ri, rv)
+    invariants(wl, si)
+    rows = sample_rows(wl, 40)
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_dense_rows(wl, rows, si[sel].cpu().numpy(), sv[sel].cpu().numpy()).assert_ok()
+
+
+def test_stream_increasing_scores_every_key_appended():
+    # Scores grow with the key index, so every key beats the running threshold.
+    L, H, d = 10000, 8, 128
+    wl = make_workload(seq_lens=[L], queries="all", H=H, B=64, m=8, k=300, seed=2,
+                       needles=False)
+    u = np.zeros(d, np.float32)
+    u[:4] = 0.5
+    K = (np.arange(1, L + 1, dtype=np.float32)[:, None] / L) * u[None, :]
+    q = np.broadcast_to(u, (L, H, d)).astype(np.float32)
+    wl = dataclasses.replace(wl, K_bits=f32_to_bf16_bits(K), q_bits=f32_to_bf16_bits(q),
+                             w=np.full((L, H), 0.5, np.float32))
+    si, sv, ri, rv, heads = run_both(wl)
+    same_sets(si, sv, ri, rv)
+    invariants(wl, si)
+    rows = [0, 299, 300, 5000, L - 1]
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_misa_rows(wl, rows, si[sel].cpu().numpy(), sv[sel].cpu().numpy(),
+                           heads=heads[sel].cpu().numpy()).assert_ok()
+
+
+def test_stream_exact_ties_resolve_to_lower_index():
+    # Keys and queries on a coarse grid: many exactly equal scores, incl. zeros.
+    L, H, d = 9600, 8, 128
+    rng = np.random.default_rng(4)
+    wl = make_workload(seq_lens=[L], queries="all", H=H, B=64, m=8, k=700, seed=3,
+                       needles=False)
+    K = rng.integers(-1, 2, size=(L, d)).astype(np.float32)
+    K[:, 2:] = 0
+    q = np.zeros((L, H, d), np.float32)
+    q[:, :, :2] = rng.integers(-1, 2, size=(L, H, 2))
+    wl = dataclasses.replace(wl, K_bits=f32_to_bf16_bits(K), q_bits=f32_to_bf16_bits(q),
+                             w=np.full((L, H), 0.25, np.float32))
+    si, sv, ri, rv, heads = run_both(wl)
+    same_sets(si, sv, ri, rv)
+    invariants(wl, si)
+    rows = sample_rows(wl, 30)
+    sel = torch.tensor(rows, device="cuda")
+    hs = heads[sel].cpu().numpy()
+    # exact ties: the selected set must equal the oracle's exactly (no tolerance games)
+    Kf = oracle.widen_bf16(wl.K_bits)
+    for j, i in enumerate(rows):
+        t = int(wl.q_pos[i])
+        I = oracle.token_scores(oracle.widen_bf16(wl.q_bits[i])[hs[j]],
+                                wl.w[i][hs[j]].astype(np.float64), Kf[:t + 1])
+        ref, _ = oracle.topk(I, wl.k)
+        assert set(si[i].tolist()) == set(ref.tolist()), f"row {i}"
