@@ -220,6 +220,17 @@ int num_sms() {
   return n > 0 ? n : kSms;
 }
 
+// Tensor-core router: power-of-two H with enough query groups to fill the GPU.
+bool route_tc_applies(const misa_problem_t* p) {
+  const int H = p->num_heads;
+  if (H != 8 && H != 16 && H != 32 && H != 64) return false;
+  return p->num_queries / route_tc_group_size(H) >= num_sms();
+}
+
+size_t route_tc_bytes(const misa_problem_t* p) {
+  return groups_bytes(p->num_queries, p->num_seqs) + align_up(route_tc_split_bytes(p->total_blocks));
+}
+
 // Streaming (fused top-k) scorer: used when every query scores its whole
 // prefix in groups that fill the GPU, no score rows are requested, and m fits.
 struct StreamPlan {
@@ -331,6 +342,7 @@ size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_
   const int T = p->num_queries, S = p->num_seqs;
   const int64_t ld = row_ld(p);
   size_t need = groups_bytes(T, S);  // router
+  if (route_tc_applies(p) && route_tc_bytes(p) > need) need = route_tc_bytes(p);
   // score / dense: chunk so the score buffer stays near kScoreBufferCap
   int64_t chunk = T;
   if ((size_t)chunk * ld * 4 > kScoreBufferCap) chunk = (int64_t)(kScoreBufferCap / ((size_t)ld * 4));
@@ -394,8 +406,17 @@ int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const
     return MISA_ERR_WORKSPACE_TOO_SMALL;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int G = route_group_size(p->num_heads);
   Carve c = carve(ws, T, S);
+  if (route_tc_applies(p) && ws_bytes >= route_tc_bytes(p)) {
+    const int G = route_tc_group_size(p->num_heads);
+    if ((rc = launch_plan_groups(*p, 0, T, G, c.groups, c.count, st))) return rc;
+    RouteTcArgs a;
+    a.p = p; a.q = q; a.w = w; a.K = K; a.Kbar = Kbar; a.m = m; a.heads = heads; a.q_r = q_r;
+    a.w_r = w_r; a.router_scores = router_scores; a.groups = c.groups; a.group_count = c.count;
+    a.max_groups = (T + G - 1) / G + S; a.split = c.buf;
+    return launch_route_tc(a, st);
+  }
+  const int G = route_group_size(p->num_heads);
   if ((rc = launch_plan_groups(*p, 0, T, G, c.groups, c.count, st))) return rc;
   return launch_route(*p, q, w, K, Kbar, m, heads, q_r, w_r, router_scores, c.groups, c.count,
                       (T + G - 1) / G + S, G, st);

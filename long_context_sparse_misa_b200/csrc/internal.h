@@ -54,6 +54,27 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
                  int max_groups, int G, cudaStream_t st);
 int route_group_size(int H);
 
+// ---- route_tc.cu: the router as a tcgen05 GEMM (prefill-sized problems).
+struct RouteTcArgs {
+  const misa_problem_t* p;
+  const uint16_t* q;
+  const float* w;
+  const uint16_t* K;
+  const float* Kbar;
+  int m;
+  int32_t* heads;
+  uint16_t* q_r;
+  float* w_r;
+  float* router_scores;
+  const int4* groups;     // route_tc_group_size(H) queries per group
+  const int* group_count;
+  int max_groups;
+  void* split;            // route_tc_split_bytes(total_blocks) of workspace
+};
+int launch_route_tc(const RouteTcArgs& a, cudaStream_t st);
+int route_tc_group_size(int H);
+size_t route_tc_split_bytes(int64_t total_blocks);
+
 // ---- score.cu
 // I[(t - q_lo) * ld + s] = sum_{j<m} wsel[t,j] ReLU(qsel[t,j] . K[key(t,s)]) for the
 // queries of the groups.  Contiguous mode (cand == nullptr): s = 0..q_pos[t].

@@ -1,0 +1,452 @@
+// Block-pooled head router on tcgen05 tensor cores.
+//
+// "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference",
+// gist.science summary, "Methodologie: MISA" (Lightweight Block-Pooled
+// Router): per-head affinities against the mean-pooled key blocks,
+// aggregated into one importance score per head; the top-h heads are kept.
+// Reading of the aggregation (as in route.cu):
+//     r[t,h] = w[t,h] * sum_{b < M_t} ReLU(q[t,h] . Kbar_t[b])
+// over the floor((t+1)/B) full blocks plus the causal partial block.
+//
+// In prefill this is a GEMM: rows (t,h) of q against the pooled keys, then a
+// ReLU-sum along the block axis.  One CTA takes a group of G queries (G*H <=
+// 512 rows, same sequence): A = its q rows (resident, 128-byte swizzle), B =
+// 128-block chunks of the pooled keys streamed by TMA, and four TMEM
+// accumulators of 128 rows x 128 blocks (all 512 columns).  The fp32 pooled
+// keys enter as a bf16 pair hi = bf16(Kbar), lo = bf16(Kbar - hi)
+// accumulated into the same fp32 accumulator, which keeps ~16 mantissa bits
+// of the pooled keys.  Epilogue warps own one row of each accumulator per
+// lane, so the block-axis ReLU-sum is inside the thread; an accumulator is
+// released as soon as it is copied to registers.
+#include "common.cuh"
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int kThreads = 192;          // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kRows = 512;             // q rows per CTA (4 accumulators of 128)
+constexpr int kChunk = 128;            // pooled blocks per chunk (accumulator columns)
+constexpr int kStages = 2;             // each stage: one of hi/lo for one chunk (2048 MMA cycles)
+constexpr int kStageBytes = kChunk * kD * 2;          // 32 KB
+constexpr int kHalfBytes = kStageBytes / 2;
+constexpr int kQHalfBytes = kRows * 128;              // 64 KB per 64-dim half
+constexpr int kQBytes = 2 * kQHalfBytes;
+constexpr int kMaxG = 16;                             // queries per group
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kMaxG * kD * 4 /*P*/ +
+                           kRows * 4 /*r*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
+
+struct Smem {
+  uint8_t* q;
+  uint8_t* k;
+  float* P;   // [kMaxG][128] causal partial-block means
+  float* r;   // [kRows] router scores of the group
+  int* pos;
+  int* flags;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;  // [4]
+  uint64_t* qfull;
+  uint64_t* drain;
+  uint32_t* tmem_slot;
+  int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* p =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.q = p;
+  s.k = p + kQBytes;
+  s.P = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
+  s.r = s.P + kMaxG * kD;
+  s.pos = reinterpret_cast<int*>(s.r + kRows);
+  s.flags = s.pos + kMaxG;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = s.tfull + 1;
+  s.qfull = s.tempty + 4;
+  s.drain = s.qfull + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
+  return s;
+}
+
+// Kbar (fp32) -> hi, lo (bf16) with hi + lo ~= Kbar.
+__global__ void split_kbar_kernel(const float* __restrict__ Kbar, int64_t n,
+                                  __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float x = Kbar[i];
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  hi[i] = h;
+  lo[i] = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
+template <int H>
+__global__ void __launch_bounds__(kThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap himap,
+                    const __grid_constant__ CUtensorMap lomap, const uint16_t* __restrict__ q,
+                    const float* __restrict__ w, const uint16_t* __restrict__ K,
+                    const int64_t* __restrict__ ko, const int64_t* __restrict__ bo,
+                    const int32_t* __restrict__ q_pos, const int4* __restrict__ groups,
+                    const int* __restrict__ group_count, int B, int m,
+                    int32_t* __restrict__ heads, uint16_t* __restrict__ q_r,
+                    float* __restrict__ w_r, float* __restrict__ router_scores,
+                    uint32_t* status) {
+  constexpr int G = (kRows / H) < kMaxG ? (kRows / H) : kMaxG;
+  constexpr int ROWS = G * H;                       // rows used (<= 512)
+  constexpr int NSUB = (ROWS + 127) / 128;          // accumulators used
+  extern __shared__ uint8_t smem_raw[];
+
+  const int gi = blockIdx.x;
+  if (gi >= *group_count) return;
+  const int4 grp = groups[gi];
+  const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
+  if (grp.w < 0 || nq <= 0) {
+    // no valid query: deterministic padding for every row of the group
+    for (int i = threadIdx.x; i < nq * m; i += blockDim.x) {
+      heads[(int64_t)qb * m + i] = -1;
+      w_r[(int64_t)qb * m + i] = 0.f;
+    }
+    for (int i = threadIdx.x; i < nq * m * (kD / 8); i += blockDim.x)
+      reinterpret_cast<uint4*>(q_r + (int64_t)qb * m * kD)[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const int64_t L = ko[seq + 1] - ko[seq];
+  const int64_t blk0 = bo[seq];
+  const int max_full = (grp.w + 1) / B;
+  const int nchunks = (max_full + kChunk - 1) / kChunk;
+
+  Smem s = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    mbar_init(s.tfull, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.tempty[i], 4);
+    mbar_init(s.qfull, 1);
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp >= 2 && threadIdx.x - 64 < kMaxG) {
+    const int qi = threadIdx.x - 64;
+    int p = -1;
+    if (qi < nq) {
+      p = q_pos[qb + qi];
+      if (p < 0 || p >= L) p = -1;
+    }
+    s.pos[qi] = p;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      mbar_arrive_expect_tx(s.qfull, 2u * ((ROWS + 31) / 32) * 32u * 128u);
+      for (int h = 0; h < 2; ++h)
+        for (int r0 = 0; r0 < ROWS; r0 += 32)
+          tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64, qb * H + r0);
+      int it = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        for (int part = 0; part < 2; ++part, ++it) {
+          const int st = it % kStages;
+          if (!mbar_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, s.abort, status)) {
+            c = nchunks;
+            break;
+          }
+          mbar_arrive_expect_tx(&s.full[st], kStageBytes);
+          const CUtensorMap* mp = part == 0 ? &himap : &lomap;
+          const int32_t row = (int32_t)(blk0 + (int64_t)c * kChunk);
+          uint8_t* dst = s.k + st * kStageBytes;
+          tma_load_2d(mp, &s.full[st], dst, 0, row);
+          tma_load_2d(mp, &s.full[st], dst + kHalfBytes, 64, row);
+        }
+      }
+      for (int i = max(0, it - kStages); i < it; ++i)
+        mbar_wait(&s.full[i % kStages], (i / kStages) & 1, s.abort, status, kDrainCycles, true);
+      mbar_wait(s.qfull, 0, s.abort, status, kDrainCycles, true);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, kChunk);
+      const uint32_t q_addr = smem_u32(s.q);
+      bool ok = mbar_wait(s.qfull, 0, s.abort, status);
+      tc_fence_after();
+      int it = 0;
+      for (int c = 0; ok && c < nchunks; ++c) {
+        for (int part = 0; ok && part < 2; ++part, ++it) {
+          const int st = it % kStages;
+          if (!(ok = mbar_wait(&s.full[st], (it / kStages) & 1, s.abort, status))) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(s.k + st * kStageBytes);
+#pragma unroll
+          for (int sub = 0; sub < NSUB; ++sub) {
+            if (part == 0 &&
+                !(ok = mbar_wait(&s.tempty[sub], (c & 1) ^ 1, s.abort, status)))
+              break;
+            if (part == 0) tc_fence_after();
+            const uint32_t d = tmem_base + sub * kChunk;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;
+              const uint64_t a = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes +
+                                                   sub * 128 * 128 + off);
+              const uint64_t b = sw128_kmajor_desc(k_addr + (kk >> 2) * kHalfBytes + off);
+              umma_bf16(d, a, b, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&s.empty[st]);
+        }
+        if (ok) umma_commit(s.tfull);
+      }
+      umma_commit(s.drain);
+      mbar_wait(s.drain, 0, s.abort, status, kDrainCycles, true);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;            // 0..127
+    const int quarter = warp & 3;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+
+    // Causal partial-block means P[qi] (mean of keys floor((t+1)/B)*B .. t),
+    // thread = dimension; overlaps the first chunks' MMAs.
+    {
+      const int d = et;
+      const uint16_t* Kseq = K + ko[seq] * kD + d;
+      bool consec = true;
+      for (int qi = 1; qi < nq; ++qi) consec &= (s.pos[qi] == s.pos[0] + qi) && s.pos[qi] >= 0;
+      consec &= s.pos[0] >= 0;
+      if (consec) {
+        const int p0 = s.pos[0], p1 = s.pos[nq - 1];
+        float run = 0.f;
+        for (int key = (p0 / B) * B; key <= p1; ++key) {
+          if (key % B == 0) run = 0.f;
+          run += bf16_bits_to_float(Kseq[(int64_t)key * kD]);
+          if (key >= p0) {
+            const int cntv = key - (key / B) * B + 1;
+            s.P[(key - p0) * kD + d] = run / (float)cntv;
+          }
+        }
+      } else {
+        for (int qi = 0; qi < nq; ++qi) {
+          const int p = s.pos[qi];
+          if (p < 0 || (p + 1) % B == 0) continue;
+          const int f = (p + 1) / B * B;
+          float run = 0.f;
+          for (int key = f; key <= p; ++key) run += bf16_bits_to_float(Kseq[(int64_t)key * kD]);
+          s.P[qi * kD + d] = run / (float)(p + 1 - f);
+        }
+      }
+    }
+
+    // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
+    // of every accumulator.
+    float acc[NSUB];
+    int lim[NSUB];
+#pragma unroll
+    for (int sub = 0; sub < NSUB; ++sub) {
+      acc[sub] = 0.f;
+      const int row = sub * 128 + quarter * 32 + lane;
+      const int qi = row / H;
+      const int p = (row < ROWS && qi < nq) ? s.pos[qi] : -1;
+      lim[sub] = (p + 1) / B;  // number of full blocks visible to this row
+    }
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      if (!(ok = warp_wait(s.tfull, c & 1, s.abort, status))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < NSUB; ++sub) {
+        float v[4][32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld32(lane_addr + sub * kChunk + j * 32, v[j]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) reg_fence32(v[j]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.tempty[sub]);
+        const int nvis = lim[sub] - c * kChunk;  // visible columns of this chunk
+        if (nvis >= kChunk) {
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+              a0 += fmaxf(v[j][x], 0.f);
+              a1 += fmaxf(v[j][x + 1], 0.f);
+            }
+          acc[sub] += a0 + a1;
+        } else if (nvis > 0) {
+          float a0 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (j * 32 + x < nvis) a0 += fmaxf(v[j][x], 0.f);
+          acc[sub] += a0;
+        }
+      }
+    }
+
+    // Epilogue threads sync on named barrier 1 (only these 128 threads).
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok) {
+#pragma unroll
+      for (int sub = 0; sub < NSUB; ++sub) {
+        const int row = sub * 128 + quarter * 32 + lane;
+        if (row >= ROWS) continue;
+        const int qi = row / H, h = row - qi * H;
+        float r = -INFINITY;
+        if (qi < nq && s.pos[qi] >= 0) {
+          const int p = s.pos[qi];
+          float total = acc[sub];
+          if ((p + 1) % B != 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)(qb + qi) * H + h) * kD);
+            const float* Pq = s.P + qi * kD;
+            float dp = 0.f;
+#pragma unroll
+            for (int i = 0; i < kD / 8; ++i) {
+              const uint4 u = __ldg(src + i);
+              dp = fmaf(__uint_as_float(u.x << 16), Pq[8 * i + 0], dp);
+              dp = fmaf(__uint_as_float(u.x & 0xFFFF0000u), Pq[8 * i + 1], dp);
+              dp = fmaf(__uint_as_float(u.y << 16), Pq[8 * i + 2], dp);
+              dp = fmaf(__uint_as_float(u.y & 0xFFFF0000u), Pq[8 * i + 3], dp);
+              dp = fmaf(__uint_as_float(u.z << 16), Pq[8 * i + 4], dp);
+              dp = fmaf(__uint_as_float(u.z & 0xFFFF0000u), Pq[8 * i + 5], dp);
+              dp = fmaf(__uint_as_float(u.w << 16), Pq[8 * i + 6], dp);
+              dp = fmaf(__uint_as_float(u.w & 0xFFFF0000u), Pq[8 * i + 7], dp);
+            }
+            total += fmaxf(dp, 0.f);
+          }
+          r = __ldg(w + (int64_t)(qb + qi) * H + h) * total;
+          if (router_scores) router_scores[(int64_t)(qb + qi) * H + h] = r;
+          if (r != r) {
+            set_status(status, MISA_STATUS_BAD_INPUT);
+            r = -INFINITY;
+          }
+        }
+        s.r[row] = r;
+      }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok) {
+      // Top-m per query by (r desc, head asc): rank of each head.
+#pragma unroll
+      for (int sub = 0; sub < NSUB; ++sub) {
+        const int row = sub * 128 + quarter * 32 + lane;
+        if (row >= ROWS) continue;
+        const int qi = row / H, h = row - qi * H;
+        if (qi >= nq) continue;
+        const int64_t t = qb + qi;
+        if (s.pos[qi] < 0) {
+          if (h < m) {
+            heads[t * m + h] = -1;
+            w_r[t * m + h] = 0.f;
+            uint4* dst = reinterpret_cast<uint4*>(q_r + (t * m + h) * kD);
+            for (int i = 0; i < kD / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          }
+          continue;
+        }
+        const float r = s.r[row];
+        const float* rq = s.r + qi * H;
+        int rank = 0;
+#pragma unroll 8
+        for (int o = 0; o < H; ++o) {
+          const float ro = rq[o];
+          rank += (ro > r) || (ro == r && o < h);
+        }
+        if (rank < m) {
+          heads[t * m + rank] = h;
+          w_r[t * m + rank] = __ldg(w + t * H + h);
+          const uint4* src = reinterpret_cast<const uint4*>(q + (t * H + h) * kD);
+          uint4* dst = reinterpret_cast<uint4*>(q_r + (t * m + rank) * kD);
+#pragma unroll
+          for (int i = 0; i < kD / 8; ++i) dst[i] = __ldg(src + i);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int H>
+int launch_h(const RouteTcArgs& a, const CUtensorMap& qmap, const CUtensorMap& himap,
+             const CUtensorMap& lomap, cudaStream_t st) {
+  auto kern = route_tc_kernel<H>;
+  int rc = set_smem_limit((const void*)kern, kSmemBytes);
+  if (rc) return rc;
+  ProfScope ps("route", st);
+  kern<<<a.max_groups, kThreads, kSmemBytes, st>>>(
+      qmap, himap, lomap, a.q, a.w, a.K, a.p->key_offsets, a.p->block_offsets, a.p->q_pos,
+      a.groups, a.group_count, a.p->block, a.m, a.heads, a.q_r, a.w_r, a.router_scores,
+      status_ptr());
+  return cuda_fail(cudaGetLastError(), "route_tc_kernel");
+}
+
+}  // namespace
+
+int route_tc_group_size(int H) {
+  const int g = kRows / H;
+  return g < kMaxG ? g : kMaxG;
+}
+
+size_t route_tc_split_bytes(int64_t total_blocks) {
+  return (size_t)total_blocks * kD * 2 * 2;  // hi + lo bf16
+}
+
+int launch_route_tc(const RouteTcArgs& a, cudaStream_t st) {
+  const misa_problem_t& p = *a.p;
+  if (a.max_groups <= 0) return MISA_OK;
+  const int64_t n = p.total_blocks * kD;
+  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.split);
+  __nv_bfloat16* lo = hi + n;
+  if (n > 0) {
+    ProfScope ps("route_split", st);
+    split_kbar_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.Kbar, n, hi, lo);
+    int rc = cuda_fail(cudaGetLastError(), "split_kbar_kernel");
+    if (rc) return rc;
+  }
+  CUtensorMap qmap, himap, lomap;
+  int rc = make_kmajor_map(&qmap, a.q, (int64_t)p.num_queries * p.num_heads, 32);
+  if (rc) return rc;
+  if ((rc = make_kmajor_map(&himap, hi, p.total_blocks, kChunk))) return rc;
+  if ((rc = make_kmajor_map(&lomap, lo, p.total_blocks, kChunk))) return rc;
+  switch (p.num_heads) {
+    case 8: return launch_h<8>(a, qmap, himap, lomap, st);
+    case 16: return launch_h<16>(a, qmap, himap, lomap, st);
+    case 32: return launch_h<32>(a, qmap, himap, lomap, st);
+    case 64: return launch_h<64>(a, qmap, himap, lomap, st);
+    default:
+      set_error("tensor-core router needs H in {8,16,32,64}, got %d", p.num_heads);
+      return MISA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace misa
