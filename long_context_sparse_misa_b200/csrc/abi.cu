@@ -182,6 +182,9 @@ int64_t row_ld(const misa_problem_t* p) { return ((int64_t)p->max_seq_len + 3) /
 
 size_t groups_bytes(int nq, int S) { return align_up(sizeof(int4) * (size_t)(nq + S) + 16); }
 
+// Failure counter (16 bytes) and list (one int per query), 256-byte aligned.
+size_t fail_bytes(int nq) { return align_up(16 + sizeof(int32_t) * (size_t)nq); }
+
 struct Carve {
   int4* groups;
   int* count;
@@ -250,7 +253,8 @@ StreamPlan stream_plan(const misa_problem_t* p, int m, int k, bool want_rows) {
   if ((T / sp.G) < 2 * sms) return sp;  // too few groups: split the keys instead
   sp.grid = sms < sp.max_groups ? sms : sp.max_groups;
   sp.cap = stream_subcap(p->max_seq_len);
-  sp.bytes = groups_bytes(T, p->num_seqs) + align_up(stream_cand_bytes(sp.grid, sp.cap));
+  sp.bytes = groups_bytes(T, p->num_seqs) + fail_bytes(T) +
+             align_up(stream_cand_bytes(sp.grid, sp.cap));
   sp.use = true;
   return sp;
 }
@@ -268,7 +272,12 @@ int score_topk_impl(const misa_problem_t* p, const uint16_t* qsel, const float* 
     StreamArgs a;
     a.p = p; a.qsel = qsel; a.wsel = wsel; a.m = m; a.K = K; a.groups = c.groups;
     a.group_count = c.count; a.max_groups = sp.max_groups; a.grid = sp.grid; a.k = k;
-    a.cand = reinterpret_cast<uint2*>(c.buf); a.subcap = sp.cap; a.idx = idx; a.val = val;
+    // workspace: group table | failure counter + list | candidate buffers
+    uint8_t* fb = reinterpret_cast<uint8_t*>(c.buf);
+    a.fail_count = reinterpret_cast<int*>(fb);
+    a.fail_list = reinterpret_cast<int32_t*>(fb + 16);
+    a.cand = reinterpret_cast<uint2*>(fb + fail_bytes(T));
+    a.subcap = sp.cap; a.idx = idx; a.val = val;
     return launch_score_stream(a, st);
   }
   const int64_t ld = scores_dbg ? scores_ld : row_ld(p);

@@ -235,6 +235,35 @@ __device__ __forceinline__ void reg_fence32(float (&v)[32]) {
                  "+f"(v[30]), "+f"(v[31]));
 }
 
+// Shared-memory reduction (no return value, shared-window address).
+__device__ __forceinline__ void red_add_shared(uint32_t* p, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Predicated memory operations: the access happens only where `pred` holds,
+// without a branch (no divergence, no reconvergence barrier).  The address
+// must be computable on every lane but is only dereferenced under `pred`.
+__device__ __forceinline__ void red_add_shared_if(uint32_t* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t@q red.shared.add.u32 [%0], 1;\n\t}\n" ::"r"(
+          smem_u32(p)),
+      "r"((int)pred)
+      : "memory");
+}
+__device__ __forceinline__ void st_global_u2_if(void* p, uint32_t x, uint32_t y, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t@q st.global.v2.u32 [%0], {%1, %2};\n\t}\n" ::"l"(
+          p),
+      "r"(x), "r"(y), "r"((int)pred)
+      : "memory");
+}
+__device__ __forceinline__ void st_global_u32_if(void* p, uint32_t x, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.u32 [%0], %1;\n\t}\n" ::"l"(p),
+      "r"(x), "r"((int)pred)
+      : "memory");
+}
+
 // a0 += w0 * r0 and a1 += w1 * r1 as one packed fp32 FMA (sm_100 f32x2).
 __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float r0,
                                       float r1) {

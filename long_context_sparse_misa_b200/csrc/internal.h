@@ -114,6 +114,8 @@ struct StreamArgs {
   int64_t subcap;         // stream_subcap(max_seq_len)
   int32_t* idx;
   float* val;
+  int32_t* fail_list;     // [T] queries whose sampled threshold did not verify
+  int* fail_count;        // device counter for fail_list
 };
 int launch_score_stream(const StreamArgs& a, cudaStream_t st);
 int stream_group_size(int m);

@@ -57,6 +57,9 @@ constexpr int kBins = 128;
 constexpr int kBinShift = 20;                    // 12-bit score key prefix: 1/8 octave
 constexpr int kHeadroom = 112;                   // bins below the first tile's maximum
 constexpr int kSelBins = 256;
+constexpr int kProbeStride = 8;                  // probe every 8th tile ...
+constexpr int kProbeOff = 4;                     // ... starting at tile 4
+constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
 
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
                            kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ + kMaxG * 4 * 4 /*wc*/ +
@@ -127,6 +130,22 @@ __device__ __forceinline__ int score_bin(uint32_t key, int base) {
   return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
 }
 
+// a[q] for a per-lane q without dynamic register indexing: a select tree
+// over the bits of q.
+template <int N>
+__device__ __forceinline__ float pick(const float (&a)[N], int q) {
+  static_assert((N & (N - 1)) == 0, "power of two");
+  float t[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) t[i] = a[i];
+#pragma unroll
+  for (int w = N / 2, bit = 0; w >= 1; w /= 2, ++bit) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = ((q >> bit) & 1) ? t[2 * i + 1] : t[2 * i];
+  }
+  return t[0];
+}
+
 // Barrier over the 8 epilogue warps (bounded; warp-uniform result).
 __device__ __forceinline__ bool ep_barrier(Smem& s, uint32_t& phase, uint32_t* status) {
   __syncwarp();
@@ -185,13 +204,17 @@ __device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint
 }
 
 // Exact top-k of one query's four candidate sub-buffers (region[r*subcap ..],
-// counts nr[r]), by one warp.  Threshold-bin entries are compacted in order
-// to the front of the region, which never overtakes the entries still to be
-// read.
-__device__ void final_select(uint2* region, int64_t subcap, const int* nr, const uint32_t* hist,
-                             int base, int k, int32_t* idx, float* val, uint32_t* selh) {
+// counts cnt[r*cstride]), by one warp.  Threshold-bin entries are compacted
+// in order to the front of the region, which never overtakes the entries
+// still to be read.
+__device__ void final_select(uint2* region, int64_t subcap, const int* cnt, int cstride,
+                             const uint32_t* hist, int base, int k, int32_t* idx, float* val,
+                             uint32_t* selh) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
+  int nr[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) nr[r] = cnt[r * cstride];
   const int n = nr[0] + nr[1] + nr[2] + nr[3];
   int out = 0;
   if (n <= k) {
@@ -212,7 +235,7 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* nr, const
     // Pass 1: entries above the threshold bin go out; threshold-bin entries
     // are compacted to the front of the region.  Each lane issues kU loads
     // before using any of them (the buffer is mostly beyond L2).
-    constexpr int kU = 8;
+    constexpr int kU = 32;
     int zpos = 0;
     for (int r = 0; r < 4; ++r) {
       const uint2* sb = region + r * subcap;
@@ -231,14 +254,13 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* nr, const
           const uint2 e = ev[u];
           const int b = j < nrr ? score_bin(order_key(__uint_as_float(e.x)), base) : -1;
           const uint32_t up = __ballot_sync(0xffffffffu, b > bstar);
-          if (b > bstar) {
-            const int o = out + __popc(up & lt);
-            idx[o] = static_cast<int32_t>(e.y);
-            val[o] = __uint_as_float(e.x) + 0.0f;
-          }
+          const int o = out + __popc(up & lt);
+          st_global_u32_if(idx + o, e.y, b > bstar && o < k);
+          st_global_u32_if(val + o, __float_as_uint(__uint_as_float(e.x) + 0.0f),
+                           b > bstar && o < k);
           out += __popc(up);
           const uint32_t zb = __ballot_sync(0xffffffffu, b == bstar);
-          if (b == bstar) region[zpos + __popc(zb & lt)] = e;
+          st_global_u2_if(region + zpos + __popc(zb & lt), e.x, e.y, b == bstar);
           zpos += __popc(zb);
         }
         __syncwarp();
@@ -293,23 +315,48 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* nr, const
   }
 }
 
+// Which group a CTA takes at schedule slot gs: longest prefix first from the
+// planner's table, or (fixup launch) one query from the failure list.
+struct Sched {
+  const int4* groups;
+  const int* count;        // number of groups (or of failed queries)
+  const int32_t* fail_in;  // fixup launch: failed query indices; else nullptr
+  int32_t* fail_out;       // first launch: where failed queries are recorded
+  int* fail_count;
+  const int32_t* qo;       // query offsets (fixup: query -> sequence)
+  const int32_t* q_pos;
+  int S;
+};
+
+__device__ __forceinline__ int4 fetch_group(const Sched& sc, int count, int gs) {
+  if (!sc.fail_in) return sc.groups[count - 1 - gs];
+  const int t = sc.fail_in[gs];
+  return make_int4(upper_segment<int32_t>(sc.qo, sc.S, t), t, t + 1, sc.q_pos[t]);
+}
+
+// Probe schedule: tiles kProbeOff, kProbeOff + kProbeStride, ... of groups
+// whose longest prefix spans at least kProbeMinTiles tiles.
+__device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
+  return (probe && ntiles >= kProbeMinTiles) ? (ntiles - kProbeOff + kProbeStride - 1) / kProbeStride
+                                             : 0;
+}
+
 template <int MH>
 __global__ void __launch_bounds__(kThreads, 1)
     score_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap qmap, const float* __restrict__ wsel,
-                        const int32_t* __restrict__ q_pos, const int64_t* __restrict__ ko,
-                        const int4* __restrict__ groups, const int* __restrict__ group_count,
-                        int k, uint2* __restrict__ cand, int64_t subcap,
-                        int32_t* __restrict__ idx_out, float* __restrict__ val_out,
-                        uint32_t* status) {
+                        const int64_t* __restrict__ ko, Sched sc, int k, uint2* __restrict__ cand,
+                        int64_t subcap, int32_t* __restrict__ idx_out,
+                        float* __restrict__ val_out, uint32_t* status) {
   constexpr int G = kN / MH;          // queries per group
   constexpr int QH = G / 2;           // queries per column half
   constexpr int QPW = QH / 2;         // queries per 64-column window
   static_assert(MH >= 8 && MH <= 64 && G <= kMaxG && QPW >= 1, "unsupported head count");
   extern __shared__ uint8_t smem_raw[];
 
-  const int count = *group_count;
+  const int count = *sc.count;
   if ((int)blockIdx.x >= count) return;
+  const bool probe = sc.fail_in == nullptr;   // the fixup launch scans without a probe
 
   Smem s = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,10 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, gl = 0;
       bool ok = true;
       for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
-        const int4 grp = groups[count - 1 - gs];
+        const int4 grp = fetch_group(sc, count, gs);
         if (grp.w < 0) continue;  // no valid query in the group
         const int64_t key_base = ko[grp.x];
         const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+        const int np = probe_tiles(probe, ntiles);
         if (!(ok = mbar_wait(s.qempty, (gl & 1) ^ 1, s.abort, status))) break;
         mbar_arrive_expect_tx(s.qfull, kQBytes);
         for (int h = 0; h < 2; ++h)
@@ -358,11 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
                         grp.y * MH + r0);
         ++gl;
-        for (int i = 0; i < ntiles; ++i, ++it) {
+        for (int step = 0; step < np + ntiles; ++step, ++it) {
+          const int tile = step < np ? kProbeOff + kProbeStride * step : step - np;
           const int st = it % kStages;
           if (!(ok = mbar_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, s.abort, status))) break;
           mbar_arrive_expect_tx(&s.full[st], kStageBytes);
-          const int32_t krow = (int32_t)(key_base + (int64_t)i * kTileKeys);
+          const int32_t krow = (int32_t)(key_base + (int64_t)tile * kTileKeys);
           uint8_t* dst = s.k + st * kStageBytes;
           tma_load_2d(&kmap, &s.full[st], dst, 0, krow);
           tma_load_2d(&kmap, &s.full[st], dst + kHalfBytes, 64, krow);
@@ -381,12 +430,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, tb = 0, gl = 0;
       bool ok = true;
       for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
-        const int4 grp = groups[count - 1 - gs];
+        const int4 grp = fetch_group(sc, count, gs);
         if (grp.w < 0) continue;
         const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+        const int np = probe_tiles(probe, ntiles);
         if (!(ok = mbar_wait(s.qfull, gl & 1, s.abort, status))) break;
         tc_fence_after();
-        for (int i = 0; i < ntiles; ++i, ++it, ++tb) {
+        for (int step = 0; step < np + ntiles; ++step, ++it, ++tb) {
           const int st = it % kStages, buf = tb & 1;
           if (!(ok = mbar_wait(&s.full[st], (it / kStages) & 1, s.abort, status))) break;
           if (!(ok = mbar_wait(&s.tempty[buf], ((tb >> 1) & 1) ^ 1, s.abort, status))) break;
@@ -422,10 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tb = 0;
     bool ok = true;
     for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
-      const int4 grp = groups[count - 1 - gs];
+      const int4 grp = fetch_group(sc, count, gs);
       if (grp.w < 0) continue;
       const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
       const int ntiles = (grp.w + kTileKeys) / kTileKeys;
+      const int np = probe_tiles(probe, ntiles);
       const int64_t L = ko[seq + 1] - ko[seq];
       // Group state: column weights, query limits, selection state.
       {
@@ -435,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (et < G) {
         int p = -1;
         if (et < nq) {
-          p = q_pos[qb + et];
+          p = sc.q_pos[qb + et];
           if (p < 0 || p >= L) p = -1;
         }
         s.pos[et] = p;
@@ -446,22 +497,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = et; i < G * kBins; i += 256) s.hist[i] = 0u;
       // This warp's slot counters (one per query; only this warp touches
       // them) and its sub-buffer of its first query; query stride 4 * subcap.
-      int* mycnt = s.wc + (half * QH) * 4 + quarter;
-      if (lane < QH) mycnt[lane * 4] = 0;
+      int* mycnt = s.wc + quarter * kMaxG + half * QH;  // [quarter][query]
+      if (lane < QH) mycnt[lane] = 0;
       uint2* mysub = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 4 * subcap +
                      (int64_t)quarter * subcap;
       const int qstride = 4 * static_cast<int>(subcap);
       if (!(ok = ep_barrier(s, ephase, status))) break;
-      float tauR[QH];  // this warp's copy of its queries' thresholds (refreshed every 4 tiles)
+      float tauR[QH];  // this warp's copy of its queries' thresholds
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) tauR[qq] = -INFINITY;
 
-      for (int i = 0; i < ntiles; ++i, ++tb) {
+      for (int step = 0; step < np + ntiles; ++step, ++tb) {
+        const bool probing = step < np;
+        const int tile = probing ? kProbeOff + kProbeStride * step : step - np;
         const int buf = tb & 1;
         if (!(ok = warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status))) break;
         tc_fence_after();
         const uint32_t taddr = lane_addr + buf * kN + half * 128;
-        float sc[QH];
+        float sc_[QH];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float v[2][32];
@@ -477,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int q2 = 0; q2 < QPW; ++q2) {
-            sc[hh * QPW + q2] = relu_wsum<MH>(
+            sc_[hh * QPW + q2] = relu_wsum<MH>(
                 [&](int j) {
                   const int col = q2 * MH + j;
                   return v[col >> 5][col & 31];
@@ -485,13 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s.w + half * 128 + hh * 64 + q2 * MH);
           }
         }
-        const int key = i * kTileKeys + lrow;
-        if (i == 0) {
-          // Anchor every query's histogram at its first tile's maximum.
+        const int key = tile * kTileKeys + lrow;
+        if (step == 0) {
+          // Anchor every query's histogram at the maximum of its first tile.
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) {
             const int qi = half * QH + qq;
-            uint32_t kk = key <= s.pos[qi] ? order_key(sc[qq]) : 0u;
+            uint32_t kk = key <= s.pos[qi] ? order_key(sc_[qq]) : 0u;
             kk = __reduce_max_sync(0xffffffffu, kk);
             if (lane == 0) atomicMax(&s.maxkey[qi], kk);
           }
@@ -500,29 +553,85 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane < QH) s.base[half * QH + lane] = hist_base(s.maxkey[half * QH + lane]);
           __syncwarp();
         }
+        if (probing) {
+          // Probe: histogram every sampled score (no appends).
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) {
+            const int qi = half * QH + qq;
+            red_add_shared_if(&s.hist[qi * kBins + score_bin(order_key(sc_[qq]), s.base[qi])],
+                              key <= s.pos[qi]);
+          }
+          if (step == np - 1) {
+            // Starting thresholds from the sample: the bin holding the r-th
+            // best sampled score, r = k*f + 4*sqrt(k*f) + 1 (f: sampled share
+            // of the query's prefix).  Verified at the end of the group.
+            if (!(ok = ep_barrier(s, ephase, status))) break;
+            for (int qi = e; qi < G; qi += kEpiWarps) {
+              const int n = s.pos[qi] + 1;
+              int ns = 0;
+              for (int j = lane; j < np; j += 32) {
+                const int rem = n - (kProbeOff + kProbeStride * j) * kTileKeys;
+                ns += rem <= 0 ? 0 : (rem > kTileKeys ? kTileKeys : rem);
+              }
+              ns = __reduce_add_sync(0xffffffffu, ns);
+              float t0 = -INFINITY;
+              if (n > k && ns > 0) {
+                const float ks = (float)k * (float)ns / (float)n;
+                const int r = (int)ceilf(ks + 4.f * sqrtf(ks)) + 1;
+                if (r <= ns) {
+                  int bstar;
+                  uint32_t A, Z;
+                  find_crossing<4>(s.hist + qi * kBins, kBins, (uint32_t)r, bstar, A, Z);
+                  if (bstar > 0)
+                    t0 = key_to_float(static_cast<uint32_t>(s.base[qi] + bstar) << kBinShift);
+                }
+              }
+              if (lane == 0) s.tau[qi] = t0;
+              for (int b = lane; b < kBins; b += 32) s.hist[qi * kBins + b] = 0u;
+            }
+            if (!(ok = ep_barrier(s, ephase, status))) break;
+#pragma unroll
+            for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
+          }
+          continue;
+        }
+        const int i = step - np;  // main-pass tile index
         if ((i & 3) == 0) {
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
         }
-        // Streaming selection: every ballot first, then the appends.
-        uint32_t bal[QH];
-#pragma unroll
-        for (int qq = 0; qq < QH; ++qq)
-          bal[qq] = __ballot_sync(0xffffffffu, key <= s.pos[half * QH + qq] && sc[qq] >= tauR[qq]);
+        // Streaming selection.  Each lane learns which of the warp's QH
+        // queries it appends to (a bit mask); the ballot, slot counter and
+        // histogram anchor of query qq live on lane qq and are fetched by
+        // shuffle.  The warp then issues one store and one histogram
+        // reduction per round, and there are as many rounds as the busiest
+        // lane has appends (usually a few), not QH.
+        uint32_t mymask = 0, balJ = 0;
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
-          if (bal[qq]) {
-            const int c0 = mycnt[qq * 4];
-            if ((bal[qq] >> lane) & 1u) {
-              const int qi = half * QH + qq;
-              mysub[qq * qstride + c0 + __popc(bal[qq] & lt)] =
-                  make_uint2(__float_as_uint(sc[qq]), static_cast<uint32_t>(key));
-              atomicAdd(&s.hist[qi * kBins + score_bin(order_key(sc[qq]), s.base[qi])], 1u);
-            }
-            __syncwarp();
-            if (lane == 0) mycnt[qq * 4] = c0 + __popc(bal[qq]);
-          }
+          const bool take = key <= s.pos[half * QH + qq] && sc_[qq] >= tauR[qq];
+          const uint32_t bq = __ballot_sync(0xffffffffu, take);
+          mymask |= (take ? 1u : 0u) << qq;
+          balJ = lane == qq ? bq : balJ;
         }
+        int c0J = 0, bsJ = 0;
+        if (lane < QH) {
+          c0J = mycnt[lane];
+          bsJ = s.base[half * QH + lane];
+        }
+        while (__any_sync(0xffffffffu, mymask != 0)) {
+          const bool act = mymask != 0;
+          const int q = act ? __ffs(mymask) - 1 : 0;
+          mymask &= mymask - 1u;
+          const uint32_t bq = __shfl_sync(0xffffffffu, balJ, q);
+          const int cq = __shfl_sync(0xffffffffu, c0J, q);
+          const int baseq = __shfl_sync(0xffffffffu, bsJ, q);
+          const float v = pick<QH>(sc_, q);
+          st_global_u2_if(mysub + q * qstride + cq + __popc(bq & lt), __float_as_uint(v),
+                          static_cast<uint32_t>(key), act);
+          red_add_shared_if(&s.hist[(half * QH + q) * kBins + score_bin(order_key(v), baseq)], act);
+        }
+        if (lane < QH) mycnt[lane] = c0J + __popc(balJ);
         // Owner warps raise tau for their queries (qi % 8 == e), every 4th tile.
         if ((i & 3) == 3) {
           for (int qi = e; qi < G; qi += kEpiWarps) {
@@ -548,8 +657,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           continue;
         }
+        // Verify the probe threshold: every key scoring at least the first
+        // threshold was appended, so min(k, n) appended entries prove that the
+        // exact top-k is among them.  Otherwise hand the query to the fixup.
+        const int napp = s.wc[qi] + s.wc[kMaxG + qi] + s.wc[2 * kMaxG + qi] +
+                         s.wc[3 * kMaxG + qi];
+        const int need = min(k, s.pos[qi] + 1);
+        if (napp < need) {
+          if (lane == 0 && sc.fail_out) sc.fail_out[atomicAdd(sc.fail_count, 1)] = t;
+          continue;
+        }
         uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 4 * subcap;
-        final_select(region, subcap, s.wc + qi * 4, s.hist + qi * kBins,
+        final_select(region, subcap, s.wc + qi, kMaxG, s.hist + qi * kBins,
                      s.base[qi], k, idx_out + (int64_t)t * k,
                      val_out + (int64_t)t * k, s.sel + e * kSelBins);
       }
@@ -568,15 +687,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int MH>
 int launch_one(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap,
-               cudaStream_t st) {
+               const Sched& sc, cudaStream_t st) {
   auto kern = score_stream_kernel<MH>;
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
-  ProfScope ps("score", st);
-  kern<<<a.grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.wsel, a.p->q_pos, a.p->key_offsets,
-                                            a.groups, a.group_count, a.k, a.cand, a.subcap,
-                                            a.idx, a.val, status_ptr());
+  ProfScope ps(sc.fail_in ? "score_fixup" : "score", st);
+  kern<<<a.grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.wsel, a.p->key_offsets, sc, a.k,
+                                            a.cand, a.subcap, a.idx, a.val, status_ptr());
   return cuda_fail(cudaGetLastError(), "score_stream_kernel");
+}
+
+template <int MH>
+int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                cudaStream_t st) {
+  Sched sc;
+  sc.groups = a.groups;
+  sc.count = a.group_count;
+  sc.fail_in = nullptr;
+  sc.fail_out = a.fail_list;
+  sc.fail_count = a.fail_count;
+  sc.qo = a.p->query_offsets;
+  sc.q_pos = a.p->q_pos;
+  sc.S = a.p->num_seqs;
+  cudaError_t e = cudaMemsetAsync(a.fail_count, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "reset failure count");
+  int rc = launch_one<MH>(a, kmap, qmap, sc, st);
+  if (rc) return rc;
+  // Queries whose probe threshold did not verify: rescan without a probe.
+  Sched fx = sc;
+  fx.fail_in = a.fail_list;
+  fx.fail_out = nullptr;
+  fx.count = a.fail_count;
+  return launch_one<MH>(a, kmap, qmap, fx, st);
 }
 
 }  // namespace
@@ -600,10 +742,10 @@ int launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   rc = make_kmajor_map(&qmap, a.qsel, (int64_t)a.p->num_queries * a.m, 32);
   if (rc) return rc;
   switch (a.m) {
-    case 8: return launch_one<8>(a, kmap, qmap, st);
-    case 16: return launch_one<16>(a, kmap, qmap, st);
-    case 32: return launch_one<32>(a, kmap, qmap, st);
-    case 64: return launch_one<64>(a, kmap, qmap, st);
+    case 8: return launch_pair<8>(a, kmap, qmap, st);
+    case 16: return launch_pair<16>(a, kmap, qmap, st);
+    case 32: return launch_pair<32>(a, kmap, qmap, st);
+    case 64: return launch_pair<64>(a, kmap, qmap, st);
     default:
       set_error("streaming scorer needs m in {8,16,32,64}, got %d", a.m);
       return MISA_ERR_UNSUPPORTED;

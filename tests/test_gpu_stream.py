@@ -149,3 +149,42 @@ def test_stream_exact_ties_resolve_to_lower_index():
                                 wl.w[i][hs[j]].astype(np.float64), Kf[:t + 1])
         ref, _ = oracle.topk(I, wl.k)
         assert set(si[i].tolist()) == set(ref.tolist()), f"row {i}"
+
+
+def test_stream_probe_overestimate_goes_through_fixup():
+    # Only the probed tiles (every 8th, from tile 4) hold high scores, and only
+    # on half their keys: the sampled threshold then admits fewer than k keys,
+    # the check fails and those queries are rescanned without a probe.
+    L, H, d = 10000, 8, 128
+    wl = make_workload(seq_lens=[L], queries="all", H=H, B=64, m=8, k=2048, seed=6,
+                       needles=False)
+    K = np.zeros((L, d), np.float32)
+    K[:, 0] = 1.0
+    s = np.arange(L)
+    high = ((s // 128) % 8 == 4) & (s % 2 == 0)
+    K[high, 0] = 10.0
+    q = np.zeros((L, H, d), np.float32)
+    q[:, :, 0] = 1.0
+    wl = dataclasses.replace(wl, K_bits=f32_to_bf16_bits(K), q_bits=f32_to_bf16_bits(q),
+                             w=np.full((L, H), 0.125, np.float32))
+    prob, Kd, qd, wd = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    misa.profile_enable(True)
+    ix.misa(qd, wd, Kd)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert "score_fixup" in prof
+    si, sv = ix.idx.clone(), ix.val.clone()
+    dbg = torch.empty((wl.T, L), dtype=torch.float32, device="cuda")
+    misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, Kd, wl.k, ix.idx, ix.val, ix.ws, dbg)
+    status_ok()
+    same_sets(si, sv, ix.idx, ix.val)
+    invariants(wl, si)
+    rows = [0, 2047, 2048, 5000, L - 1]
+    Kf = oracle.widen_bf16(wl.K_bits)
+    for i in rows:
+        I = oracle.token_scores(oracle.widen_bf16(wl.q_bits[i])[:8], wl.w[i][:8].astype(np.float64),
+                                Kf[:i + 1])
+        ref, _ = oracle.topk(I, wl.k)
+        assert set(si[i].tolist()) == set(ref.tolist()), f"row {i}"
