@@ -228,10 +228,31 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* cnt, int 
       out += nr[r];
     }
   } else {
+    // Pass 0: histogram of the entries (bins relative to the query's anchor).
+    constexpr int kH = 16;
+    for (int i = lane; i < kBins; i += 32) selh[i] = 0u;
+    __syncwarp();
+    for (int r = 0; r < 4; ++r) {
+      const uint2* sb = region + r * subcap;
+      for (int j0 = 0; j0 < nr[r]; j0 += 32 * kH) {
+        uint32_t xv[kH];
+#pragma unroll
+        for (int u = 0; u < kH; ++u) {
+          const int j = j0 + u * 32 + lane;
+          xv[u] = j < nr[r] ? __ldcs(&sb[j].x) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kH; ++u)
+          red_add_shared_if(&selh[score_bin(order_key(__uint_as_float(xv[u])), base)],
+                            j0 + u * 32 + lane < nr[r]);
+      }
+    }
+    __syncwarp();
     int bstar;
     uint32_t A, Z;
     find_crossing<4>(hist, kBins, (uint32_t)k, bstar, A, Z);
     uint32_t need = (uint32_t)k - A;
+    __syncwarp();
     // Pass 1: entries above the threshold bin go out; threshold-bin entries
     // are compacted to the front of the region.  Each lane issues kU loads
     // before using any of them (the buffer is mostly beyond L2).
@@ -491,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         s.pos[et] = p;
         s.row[et] = qb + et;
-        s.tau[et] = -INFINITY;
+        s.tau[et] = p >= 0 ? -INFINITY : INFINITY;  // padding / invalid slots never append
         s.maxkey[et] = 0u;
       }
       for (int i = et; i < G * kBins; i += 256) s.hist[i] = 0u;
@@ -503,6 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      (int64_t)quarter * subcap;
       const int qstride = 4 * static_cast<int>(subcap);
       if (!(ok = ep_barrier(s, ephase, status))) break;
+      int minpos = 0x7fffffff;  // smallest valid position of the group (-1 if any invalid)
+      for (int qi = 0; qi < nq; ++qi) minpos = min(minpos, s.pos[qi]);
       float tauR[QH];  // this warp's copy of its queries' thresholds
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) tauR[qq] = -INFINITY;
@@ -574,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ns += rem <= 0 ? 0 : (rem > kTileKeys ? kTileKeys : rem);
               }
               ns = __reduce_add_sync(0xffffffffu, ns);
-              float t0 = -INFINITY;
+              float t0 = s.pos[qi] >= 0 ? -INFINITY : INFINITY;
               if (n > k && ns > 0) {
                 const float ks = (float)k * (float)ns / (float)n;
                 const int r = (int)ceilf(ks + 4.f * sqrtf(ks)) + 1;
@@ -607,44 +630,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         // reduction per round, and there are as many rounds as the busiest
         // lane has appends (usually a few), not QH.
         uint32_t mymask = 0, balJ = 0;
+        // tiles wholly below every query's position need no causal compare
+        const bool full_tile = (tile + 1) * kTileKeys <= minpos + 1;
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
-          const bool take = key <= s.pos[half * QH + qq] && sc_[qq] >= tauR[qq];
+          const bool take = (full_tile || key <= s.pos[half * QH + qq]) && sc_[qq] >= tauR[qq];
           const uint32_t bq = __ballot_sync(0xffffffffu, take);
           mymask |= (take ? 1u : 0u) << qq;
           balJ = lane == qq ? bq : balJ;
         }
-        int c0J = 0, bsJ = 0;
-        if (lane < QH) {
-          c0J = mycnt[lane];
-          bsJ = s.base[half * QH + lane];
-        }
+        int c0J = lane < QH ? mycnt[lane] : 0;
         while (__any_sync(0xffffffffu, mymask != 0)) {
           const bool act = mymask != 0;
           const int q = act ? __ffs(mymask) - 1 : 0;
           mymask &= mymask - 1u;
           const uint32_t bq = __shfl_sync(0xffffffffu, balJ, q);
           const int cq = __shfl_sync(0xffffffffu, c0J, q);
-          const int baseq = __shfl_sync(0xffffffffu, bsJ, q);
           const float v = pick<QH>(sc_, q);
           st_global_u2_if(mysub + q * qstride + cq + __popc(bq & lt), __float_as_uint(v),
                           static_cast<uint32_t>(key), act);
-          red_add_shared_if(&s.hist[(half * QH + q) * kBins + score_bin(order_key(v), baseq)], act);
         }
         if (lane < QH) mycnt[lane] = c0J + __popc(balJ);
-        // Owner warps raise tau for their queries (qi % 8 == e), every 4th tile.
-        if ((i & 3) == 3) {
-          for (int qi = e; qi < G; qi += kEpiWarps) {
-            int bstar;
-            uint32_t A, Z;
-            find_crossing<4>(s.hist + qi * kBins, kBins, (uint32_t)k, bstar, A, Z);
-            if (lane == 0 && bstar > 0) {
-              const float edge =
-                  key_to_float(static_cast<uint32_t>(s.base[qi] + bstar) << kBinShift);
-              if (edge > s.tau[qi]) s.tau[qi] = edge;
-            }
-          }
-        }
       }
       if (!ok) break;
       if (!(ok = ep_barrier(s, ephase, status))) break;
@@ -668,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           continue;
         }
         uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 4 * subcap;
-        final_select(region, subcap, s.wc + qi, kMaxG, s.hist + qi * kBins,
+        final_select(region, subcap, s.wc + qi, kMaxG, s.sel + e * kSelBins,
                      s.base[qi], k, idx_out + (int64_t)t * k,
                      val_out + (int64_t)t * k, s.sel + e * kSelBins);
       }
