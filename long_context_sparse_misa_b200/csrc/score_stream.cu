@@ -21,22 +21,24 @@
 // before each wait, the TMEM buffer released after the second pair, then per
 // key and query I = sum_j w_j ReLU(acc_j), the causal mask, and the
 // streaming selection:
-//   * tau_q, a safe lower bound on query q's k-th best score: a key is
-//     appended to q's candidate buffer only if I >= tau_q.  Each (query,
-//     lane quarter) has a private sub-buffer with one slot per key the
-//     quarter can see, so nothing can overflow and the slot counter lives in
-//     a register (no returning atomics on the hot path).
-//   * a 128-bin histogram per query (1/8-octave bins of the order-preserving
-//     score key, anchored 14 octaves below the first tile's maximum) counts
-//     the appended scores; every other tile the owner warp raises tau_q to the
-//     lower edge of the bin where the count from the top reaches k.  At least
-//     k appended scores are >= that edge, so a later key scoring below it
-//     cannot be in the top-k whatever its index; equal scores are kept, so
-//     ties resolved by token index stay exact.  Reads of the histogram race
-//     with other warps' appends only towards a lower (still safe) tau.
-//   * at the end of the group the owner warp selects exactly: entries above
-//     the histogram's threshold bin are taken, the threshold bin is resolved
-//     by a warp-level radix select over (score, lower index first).
+//   * probe: a group first scores every 8th tile of its prefix and keeps a
+//     128-bin histogram per query (1/8-octave bins of the order-preserving
+//     score key, anchored 14 octaves below the first scored tile's maximum).
+//     The starting threshold tau_q is the lower edge of the bin holding the
+//     r-th best sampled score, r = k*f + 4*sqrt(k*f) + 1 (f = sampled share
+//     of the prefix), i.e. a few standard deviations below the expected k-th
+//     best score.
+//   * main pass over all tiles: a key is appended to query q's candidates
+//     only if I >= tau_q.  Each (query, lane quarter) has a private
+//     sub-buffer with one slot per key the quarter can see, so nothing can
+//     overflow; slot ranks come from per-query ballots, and each lane issues
+//     its appends in rounds (as many rounds as the busiest lane has appends).
+//   * check and select: every key scoring at least tau_q was appended, so if
+//     at least min(k, n) keys were appended the exact top-k is among them.
+//     The owner warp then histograms the candidates, takes those above the
+//     bin holding the k-th, and resolves that bin with a warp-level radix
+//     select over (score, lower index first).  A query with too few
+//     candidates is listed and rescanned by a second launch without a probe.
 #include "common.cuh"
 #include "internal.h"
 
