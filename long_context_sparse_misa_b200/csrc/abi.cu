@@ -125,6 +125,13 @@ cudaEvent_t take_event() {
 }
 }  // namespace
 
+int num_sms() {
+  int dev = 0, n = kSms;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : kSms;
+}
+
 ProfScope::ProfScope(const char* name, cudaStream_t s) : slot(-1), st(s) {
   if (!t_prof_on) return;
   ProfRecord r{name, take_event(), take_event()};
@@ -180,7 +187,11 @@ bool pow2_le64(int x) { return x >= 1 && x <= 64 && (x & (x - 1)) == 0; }
 
 int64_t row_ld(const misa_problem_t* p) { return ((int64_t)p->max_seq_len + 3) / 4 * 4; }
 
-size_t groups_bytes(int nq, int S) { return align_up(sizeof(int4) * (size_t)(nq + S) + 16); }
+// Group table: int4 [nq + S], the count word (16 bytes), first group of each
+// sequence int [S].
+size_t groups_bytes(int nq, int S) {
+  return align_up(sizeof(int4) * (size_t)(nq + S) + 16 + sizeof(int) * (size_t)S);
+}
 
 // Failure counter (16 bytes) and list (one int per query), 256-byte aligned.
 size_t fail_bytes(int nq) { return align_up(16 + sizeof(int32_t) * (size_t)nq); }
@@ -216,18 +227,23 @@ int chunk_queries(const misa_problem_t* p, int64_t ld, size_t ws_bytes) {
   return 0;
 }
 
-int num_sms() {
-  int dev = 0, n = kSms;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : kSms;
-}
-
 // Tensor-core router: power-of-two H with enough query groups to fill the GPU.
 bool route_tc_applies(const misa_problem_t* p) {
   const int H = p->num_heads;
   if (H != 8 && H != 16 && H != 32 && H != 64) return false;
   return p->num_queries / route_tc_group_size(H) >= num_sms();
+}
+
+// CUDA-core router: group table, then the partial sums of split block ranges.
+int route_max_groups(const misa_problem_t* p) {
+  const int G = route_group_size(p->num_heads);
+  return (p->num_queries + G - 1) / G + p->num_seqs;
+}
+
+size_t route_bytes(const misa_problem_t* p) {
+  const int mg = route_max_groups(p);
+  return groups_bytes(p->num_queries, p->num_seqs) +
+         align_up(route_split_bytes(mg, route_split_count(*p, mg, num_sms())));
 }
 
 size_t route_tc_bytes(const misa_problem_t* p) {
@@ -350,7 +366,7 @@ size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_
   }
   const int T = p->num_queries, S = p->num_seqs;
   const int64_t ld = row_ld(p);
-  size_t need = groups_bytes(T, S);  // router
+  size_t need = route_bytes(p);  // router
   if (route_tc_applies(p) && route_tc_bytes(p) > need) need = route_tc_bytes(p);
   // score / dense: chunk so the score buffer stays near kScoreBufferCap
   int64_t chunk = T;
@@ -426,9 +442,13 @@ int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const
     return launch_route_tc(a, st);
   }
   const int G = route_group_size(p->num_heads);
+  const int mg = route_max_groups(p);
+  // Split the block ranges only when the workspace holds the partial sums.
+  int nsplit = route_split_count(*p, mg, num_sms());
+  if (nsplit > 1 && ws_bytes < route_bytes(p)) nsplit = 1;
   if ((rc = launch_plan_groups(*p, 0, T, G, c.groups, c.count, st))) return rc;
   return launch_route(*p, q, w, K, Kbar, m, heads, q_r, w_r, router_scores, c.groups, c.count,
-                      (T + G - 1) / G + S, G, st);
+                      mg, G, nsplit, nsplit > 1 ? c.buf : nullptr, st);
 }
 
 int misa_score_topk(const misa_problem_t* p, const uint16_t* q_r, const float* w_r, int32_t m,

@@ -29,6 +29,8 @@ uint32_t* status_ptr();
 int make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 int set_smem_limit(const void* kernel, int bytes);
+// SMs of the current device.
+int num_sms();
 
 // Tracing: brackets one kernel launch with events on `st` when profiling is on.
 struct ProfScope {
@@ -42,7 +44,8 @@ struct ProfScope {
 int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* block_offsets,
                          cudaStream_t st);
 // Build query groups of at most G queries over query rows [q_lo, q_hi).
-// groups: int4 [q_hi-q_lo + S]; count: one int.
+// groups: int4 [q_hi-q_lo + S]; count: one int, followed 16 bytes later by
+// int [S] of scratch (the first group of each sequence).
 int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
                        int* count, cudaStream_t st);
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st);
@@ -51,8 +54,12 @@ int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStr
 int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, const uint16_t* K,
                  const float* Kbar, int m, int32_t* heads, uint16_t* q_r, float* w_r,
                  float* router_scores, const int4* groups, const int* group_count,
-                 int max_groups, int G, cudaStream_t st);
+                 int max_groups, int G, int nsplit, float* partial, cudaStream_t st);
 int route_group_size(int H);
+// Pooled-block ranges per group for the CUDA-core router (1 = no split) and
+// the workspace its partial sums take.
+int route_split_count(const misa_problem_t& p, int max_groups, int sms);
+size_t route_split_bytes(int max_groups, int nsplit);
 
 // ---- route_tc.cu: the router as a tcgen05 GEMM (prefill-sized problems).
 struct RouteTcArgs {

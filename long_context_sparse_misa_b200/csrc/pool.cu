@@ -53,27 +53,26 @@ __global__ void block_offsets_kernel(const int64_t* __restrict__ ko, int S, int 
   }
 }
 
-// One CTA: split every sequence's queries (restricted to [q_lo, q_hi)) into
-// groups of at most G and record {seq, q_begin, q_end, max_pos}.  A scan over
-// sequences gives each sequence its first group index; then every warp takes
-// groups round-robin and reduces the positions of its group's queries.
-// Positions outside their sequence are flagged and left out of max_pos.
-__global__ void plan_groups_kernel(const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
-                                   const int32_t* __restrict__ q_pos, int S, int q_lo, int q_hi,
-                                   int G, int4* __restrict__ groups, int* __restrict__ count,
-                                   uint32_t* status) {
+// Query groups: every sequence's queries, restricted to [q_lo, q_hi), are cut
+// into groups of at most G, recorded as {seq, q_begin, q_end, max_pos}.
+// First a one-CTA scan over sequences gives each sequence the index of its
+// first group (first[s]) and the group count; then one warp per group finds
+// its sequence by binary search over first[] and reduces its queries'
+// positions.  Positions outside their sequence are flagged and left out of
+// max_pos.
+__global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_lo, int q_hi,
+                                  int G, int* __restrict__ first, int* __restrict__ count) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
-  __shared__ int s_first[1024], s_ng[1024], s_b[1024], s_e[1024];
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int base = 0; base < S; base += blockDim.x) {
+    const int c0 = carry;
     const int s = base + threadIdx.x;
-    int b = 0, e = 0, ng = 0;
+    int ng = 0;
     if (s < S) {
-      b = max(qo[s], q_lo);
-      e = min(qo[s + 1], q_hi);
+      const int b = max(qo[s], q_lo), e = min(qo[s + 1], q_hi);
       ng = e > b ? (e - b + G - 1) / G : 0;
     }
     int x = ng;
@@ -94,39 +93,59 @@ __global__ void plan_groups_kernel(const int64_t* __restrict__ ko, const int32_t
       warp_sums[lane] = ws;
     }
     __syncthreads();
-    const int first = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - ng;
-    s_first[threadIdx.x] = first;
-    s_ng[threadIdx.x] = ng;
-    s_b[threadIdx.x] = b;
-    s_e[threadIdx.x] = e;
+    const int f = c0 + (warp > 0 ? warp_sums[warp - 1] : 0) + x - ng;
+    if (s < S) first[s] = f;
     __syncthreads();
-    const int nseq = min((int)blockDim.x, S - base);
-    for (int j = 0; j < nseq; ++j) {
-      const int ngj = s_ng[j];
-      if (ngj == 0) continue;
-      const int sj = base + j, bj = s_b[j], ej = s_e[j], fj = s_first[j];
-      const int64_t L = ko[sj + 1] - ko[sj];
-      for (int g = warp; g < ngj; g += nwarps) {
-        const int qb = bj + g * G, qe = min(qb + G, ej);
-        int mp = -1;
-        for (int t = qb + lane; t < qe; t += 32) {
-          const int pos = q_pos[t];
-          if (pos < 0 || pos >= L) set_status(status, MISA_STATUS_BAD_INPUT);
-          else mp = max(mp, pos);
-        }
-        mp = __reduce_max_sync(0xffffffffu, mp);
-        if (lane == 0) groups[fj + g] = make_int4(sj, qb, qe, mp);
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry = first + ng;
+    if (threadIdx.x == blockDim.x - 1) carry = f + ng;
     __syncthreads();
   }
   if (threadIdx.x == 0) *count = carry;
 }
 
-// One warp per pooled row; each lane owns 4 of the 128 dims.  fp64 sums so
-// that the fp32 mean is the correctly rounded mean of the bf16 keys.
+__global__ void group_fill_kernel(const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
+                                  const int32_t* __restrict__ q_pos, int S, int q_lo, int q_hi,
+                                  int G, const int* __restrict__ first,
+                                  const int* __restrict__ count, int4* __restrict__ groups,
+                                  uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int fg = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
+  if (fg >= *count) return;
+  int lo = 0, hi = S - 1;  // last sequence j with first[j] <= fg
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (first[mid] <= fg) lo = mid; else hi = mid - 1;
+  }
+  const int j = lo;
+  const int b = max(qo[j], q_lo), e = min(qo[j + 1], q_hi);
+  const int qb = b + (fg - first[j]) * G, qe = min(qb + G, e);
+  const int64_t L = ko[j + 1] - ko[j];
+  int mp = -1;
+  for (int t = qb + lane; t < qe; t += 32) {
+    const int pos = q_pos[t];
+    if (pos < 0 || pos >= L) set_status(status, MISA_STATUS_BAD_INPUT);
+    else mp = max(mp, pos);
+  }
+  mp = __reduce_max_sync(0xffffffffu, mp);
+  if (lane == 0) groups[fg] = make_int4(j, qb, qe, mp);
+}
+
+// One warp per pooled row.  The two half-warps take alternate keys and each
+// lane owns 8 of the 128 dims (one 16-byte load per key), with 8 loads in
+// flight per lane; the halves are added at the end.  fp64 sums: every
+// partial sum of at most 4096 bf16 keys is exact for keys within 2^33 of one
+// another in magnitude, so the split does not change the result, and the
+// fp32 mean is the correctly rounded mean of the bf16 keys.
+__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 v) {
+  acc[0] += (double)__uint_as_float(v.x << 16);
+  acc[1] += (double)__uint_as_float(v.x & 0xFFFF0000u);
+  acc[2] += (double)__uint_as_float(v.y << 16);
+  acc[3] += (double)__uint_as_float(v.y & 0xFFFF0000u);
+  acc[4] += (double)__uint_as_float(v.z << 16);
+  acc[5] += (double)__uint_as_float(v.z & 0xFFFF0000u);
+  acc[6] += (double)__uint_as_float(v.w << 16);
+  acc[7] += (double)__uint_as_float(v.w & 0xFFFF0000u);
+}
+
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ K,
                                                    const int64_t* __restrict__ ko,
                                                    const int64_t* __restrict__ bo, int S, int B,
@@ -140,39 +159,40 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   const int64_t k0 = ko[s] + b * B;
   const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
   if (k0 < 0 || k1 > total_keys || k1 <= k0) {
-    set_status(status, MISA_STATUS_BOUNDS);
+    if (lane == 0) set_status(status, MISA_STATUS_BOUNDS);
     return;
   }
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  const uint2* src = reinterpret_cast<const uint2*>(K) + k0 * (kD / 4) + lane;
-  int64_t n = k1 - k0;
-  int64_t i = 0;
-  for (; i + 4 <= n; i += 4) {
-    uint2 v[4];
+  constexpr int kRow16 = kD / 8;  // 16-byte chunks per key
+  const int half = lane >> 4, hl = lane & 15;
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+  const uint4* src = reinterpret_cast<const uint4*>(K) + k0 * kRow16 + hl;
+  const int64_t n = k1 - k0;
+  int64_t i = half;
+  for (; i + 14 < n; i += 16) {  // keys i, i+2, ..., i+14
+    uint4 v[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = __ldg(src + (i + u) * (kD / 4));
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (i + 2 * u) * kRow16);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      acc[0] += (double)__uint_as_float(v[u].x << 16);
-      acc[1] += (double)__uint_as_float(v[u].x & 0xFFFF0000u);
-      acc[2] += (double)__uint_as_float(v[u].y << 16);
-      acc[3] += (double)__uint_as_float(v[u].y & 0xFFFF0000u);
-    }
+    for (int u = 0; u < 8; ++u) add_bf16x8(acc, v[u]);
   }
-  for (; i < n; ++i) {
-    const uint2 v = __ldg(src + i * (kD / 4));
-    acc[0] += (double)__uint_as_float(v.x << 16);
-    acc[1] += (double)__uint_as_float(v.x & 0xFFFF0000u);
-    acc[2] += (double)__uint_as_float(v.y << 16);
-    acc[3] += (double)__uint_as_float(v.y & 0xFFFF0000u);
+  for (; i < n; i += 2) add_bf16x8(acc, __ldg(src + i * kRow16));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
+  if (half == 0) {
+    const double cnt = (double)n;
+    float4 lo, hi;
+    lo.x = __double2float_rn(acc[0] / cnt);
+    lo.y = __double2float_rn(acc[1] / cnt);
+    lo.z = __double2float_rn(acc[2] / cnt);
+    lo.w = __double2float_rn(acc[3] / cnt);
+    hi.x = __double2float_rn(acc[4] / cnt);
+    hi.y = __double2float_rn(acc[5] / cnt);
+    hi.z = __double2float_rn(acc[6] / cnt);
+    hi.w = __double2float_rn(acc[7] / cnt);
+    float4* dst = reinterpret_cast<float4*>(Kbar) + row * (kD / 4) + 2 * hl;
+    dst[0] = lo;
+    dst[1] = hi;
   }
-  const double cnt = (double)n;
-  float4 out;
-  out.x = __double2float_rn(acc[0] / cnt);
-  out.y = __double2float_rn(acc[1] / cnt);
-  out.z = __double2float_rn(acc[2] / cnt);
-  out.w = __double2float_rn(acc[3] / cnt);
-  reinterpret_cast<float4*>(Kbar)[row * (kD / 4) + lane] = out;
 }
 
 }  // namespace
@@ -187,9 +207,16 @@ int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* bloc
 int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
                        int* count, cudaStream_t st) {
   ProfScope ps("plan_groups", st);
-  plan_groups_kernel<<<1, 1024, 0, st>>>(p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs,
-                                         q_lo, q_hi, G, groups, count, status_ptr());
-  return cuda_fail(cudaGetLastError(), "plan_groups_kernel");
+  int* first = count + 4;  // [S] after the count word (see groups_bytes)
+  group_scan_kernel<<<1, 1024, 0, st>>>(p.query_offsets, p.num_seqs, q_lo, q_hi, G, first, count);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "group_scan_kernel");
+  const int64_t max_groups = (int64_t)(q_hi - q_lo + G - 1) / G + p.num_seqs;
+  const int warps = 8;
+  group_fill_kernel<<<(unsigned)((max_groups + warps - 1) / warps), warps * 32, 0, st>>>(
+      p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo, q_hi, G, first, count, groups,
+      status_ptr());
+  return cuda_fail(cudaGetLastError(), "group_fill_kernel");
 }
 
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st) {

@@ -13,6 +13,15 @@
 // One CTA per query group (same sequence); thread = (query, head) row with
 // its q row in registers; pooled blocks are staged through shared memory and
 // read by broadcast.  fp32 arithmetic on CUDA cores.
+//
+// Decode batches have too few query groups to fill the GPU, and each group
+// scans every pooled block of a long prefix.  There the pooled blocks are
+// split into contiguous ranges, one CTA per (group, range) writes its partial
+// sums, and a second launch adds the ranges in ascending order (a fixed
+// order, so the result does not depend on scheduling), adds the causal
+// partial block, and takes the top-m.  The number of ranges is taken on the
+// device from the actual group count, so that the (group, range) CTAs form
+// one wave.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,6 +31,14 @@ namespace {
 constexpr int kRouteThreads = 256;
 constexpr int kChunk = 32;  // pooled blocks per shared-memory stage
 
+// kWhole: one CTA does everything for its group.
+// kPartial: CTA (group, y) with y < ns sums range y of the full pooled
+//           blocks; CTA (group, ns) evaluates the causal partial block.  Each
+//           stores its per-thread sum; nothing else.
+// kFinish: adds the ns + 1 stored sums in order, then ranks as kWhole.
+enum RouteMode { kWhole = 0, kPartial = 1, kFinish = 2 };
+
+template <int kMode>
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w,
                  const uint16_t* __restrict__ K, const float* __restrict__ Kbar,
@@ -29,14 +46,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
                  const int32_t* __restrict__ q_pos, const int4* __restrict__ groups,
                  const int* __restrict__ group_count, int H, int B, int m, int G,
                  int32_t* __restrict__ heads, uint16_t* __restrict__ q_r, float* __restrict__ w_r,
-                 float* __restrict__ router_scores, uint32_t* status) {
+                 float* __restrict__ router_scores, uint32_t* status, int nsplit_max,
+                 int sms, float* __restrict__ partial) {
   extern __shared__ __align__(16) float smem_f[];
   float* kb = smem_f;                         // [kChunk][128]
   float* part = kb + kChunk * kD;             // [G][128]
   float* rs = part + G * kD;                  // [G][H]
 
-  const int g = blockIdx.x;
-  if (g >= *group_count) return;
+  const int count = *group_count;
+  // Full-block ranges per group (kPartial / kFinish): as many as keep the
+  // count * (ns + 1) CTAs within one wave.
+  const int ns = kMode == kWhole ? 1 : max(1, min(nsplit_max, sms / max(count, 1) - 1));
+  const int g = kMode == kPartial ? (int)blockIdx.x / (ns + 1) : (int)blockIdx.x;
+  if (g >= count) return;
+  const int y = kMode == kPartial ? (int)blockIdx.x - g * (ns + 1) : 0;
+  const bool do_full = kMode == kWhole || (kMode == kPartial && y < ns);
+  const bool do_tail = kMode == kWhole || (kMode == kPartial && y == ns);
   const int4 grp = groups[g];
   const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
   const int tid = threadIdx.x;
@@ -52,7 +77,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   const int max_full = (grp.w + 1) / B;
 
   float qreg[kD];
-  if (valid) {
+  if (valid && kMode != kFinish) {
     const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)t * H + h) * kD);
 #pragma unroll
     for (int i = 0; i < kD / 8; ++i) {
@@ -71,63 +96,101 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     for (int i = 0; i < kD; ++i) qreg[i] = 0.f;
   }
 
-  // Full blocks: ReLU(q . Kbar_b) summed over b < nfull.
+  // Full blocks: ReLU(q . Kbar_b) summed over b < nfull (over this CTA's
+  // range of blocks when split).
   float acc = 0.f;
-  const float4* kbar4 = reinterpret_cast<const float4*>(Kbar + bo[seq] * kD);
-  for (int c0 = 0; c0 < max_full; c0 += kChunk) {
-    const int nb = min(kChunk, max_full - c0);
-    __syncthreads();
-    for (int i = tid; i < nb * (kD / 4); i += kRouteThreads)
-      reinterpret_cast<float4*>(kb)[i] = __ldg(kbar4 + (int64_t)c0 * (kD / 4) + i);
-    __syncthreads();
-    const int lim = min(nb, nfull - c0);
-    for (int b = 0; b < lim; ++b) {
-      const float4* row = reinterpret_cast<const float4*>(kb + b * kD);
-      float d0 = 0.f, d1 = 0.f;
+  if (do_full) {
+    int b_lo = 0, b_hi = max_full;
+    if (kMode == kPartial) {
+      const int range = (max_full + ns - 1) / ns;
+      b_lo = y * range;
+      b_hi = min(max_full, b_lo + range);
+    }
+    const float4* kbar4 = reinterpret_cast<const float4*>(Kbar + bo[seq] * kD);
+    for (int c0 = b_lo; c0 < b_hi; c0 += kChunk) {
+      const int nb = min(kChunk, b_hi - c0);
+      __syncthreads();
+      for (int i = tid; i < nb * (kD / 4); i += kRouteThreads)
+        reinterpret_cast<float4*>(kb)[i] = __ldg(kbar4 + (int64_t)c0 * (kD / 4) + i);
+      __syncthreads();
+      const int lim = min(nb, nfull - c0);
+      for (int b = 0; b < lim; ++b) {
+        const float4* row = reinterpret_cast<const float4*>(kb + b * kD);
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
-      for (int i = 0; i < kD / 4; i += 2) {
-        const float4 a = row[i], c = row[i + 1];
-        d0 = fmaf(qreg[4 * i + 0], a.x, d0);
-        d0 = fmaf(qreg[4 * i + 1], a.y, d0);
-        d0 = fmaf(qreg[4 * i + 2], a.z, d0);
-        d0 = fmaf(qreg[4 * i + 3], a.w, d0);
-        d1 = fmaf(qreg[4 * i + 4], c.x, d1);
-        d1 = fmaf(qreg[4 * i + 5], c.y, d1);
-        d1 = fmaf(qreg[4 * i + 6], c.z, d1);
-        d1 = fmaf(qreg[4 * i + 7], c.w, d1);
+        for (int i = 0; i < kD / 4; i += 2) {
+          const float4 a = row[i], c = row[i + 1];
+          d0 = fmaf(qreg[4 * i + 0], a.x, d0);
+          d1 = fmaf(qreg[4 * i + 1], a.y, d1);
+          d0 = fmaf(qreg[4 * i + 2], a.z, d0);
+          d1 = fmaf(qreg[4 * i + 3], a.w, d1);
+          d2 = fmaf(qreg[4 * i + 4], c.x, d2);
+          d3 = fmaf(qreg[4 * i + 5], c.y, d3);
+          d2 = fmaf(qreg[4 * i + 6], c.z, d2);
+          d3 = fmaf(qreg[4 * i + 7], c.w, d3);
+        }
+        acc += fmaxf((d0 + d1) + (d2 + d3), 0.f);
       }
-      acc += fmaxf(d0 + d1, 0.f);
+    }
+  }
+  // Causal partial block of every query of the group (mean of its visible keys).
+  if (do_tail) {
+    __syncthreads();
+    for (int i = tid; i < G * kD; i += kRouteThreads) part[i] = 0.f;
+    __syncthreads();
+    // Thread per (query, pair of dims); keys summed in order, 8 loads in flight.
+    for (int item = tid; item < nq * (kD / 2); item += kRouteThreads) {
+      const int qi = item / (kD / 2), dp = item - qi * (kD / 2);
+      const int p2 = q_pos[qb + qi];
+      if (p2 < 0 || p2 >= L) continue;
+      const int f2 = (p2 + 1) / B * B;
+      const int cnt = p2 + 1 - f2;
+      if (cnt == 0) continue;
+      const uint32_t* col = reinterpret_cast<const uint32_t*>(K + (ko[seq] + f2) * kD) + dp;
+      float s0 = 0.f, s1 = 0.f;
+      int key = 0;
+      for (; key + 8 <= cnt; key += 8) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(col + (int64_t)(key + u) * (kD / 2));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          s0 += __uint_as_float(v[u] << 16);
+          s1 += __uint_as_float(v[u] & 0xFFFF0000u);
+        }
+      }
+      for (; key < cnt; ++key) {
+        const uint32_t v = __ldg(col + (int64_t)key * (kD / 2));
+        s0 += __uint_as_float(v << 16);
+        s1 += __uint_as_float(v & 0xFFFF0000u);
+      }
+      part[qi * kD + 2 * dp] = s0 / (float)cnt;
+      part[qi * kD + 2 * dp + 1] = s1 / (float)cnt;
+    }
+    __syncthreads();
+    if (valid && nfull * B != n) {
+      const float4* row = reinterpret_cast<const float4*>(part + qq * kD);
+      float d = 0.f;
+#pragma unroll
+      for (int i = 0; i < kD / 4; ++i) {
+        const float4 a = row[i];
+        d = fmaf(qreg[4 * i + 0], a.x, d);
+        d = fmaf(qreg[4 * i + 1], a.y, d);
+        d = fmaf(qreg[4 * i + 2], a.z, d);
+        d = fmaf(qreg[4 * i + 3], a.w, d);
+      }
+      acc += fmaxf(d, 0.f);
     }
   }
 
-  // Causal partial block of every query of the group (mean of its visible keys).
-  __syncthreads();
-  for (int i = tid; i < G * kD; i += kRouteThreads) part[i] = 0.f;
-  __syncthreads();
-  for (int item = tid; item < nq * kD; item += kRouteThreads) {
-    const int qi = item / kD, dim = item - qi * kD;
-    const int p2 = q_pos[qb + qi];
-    if (p2 < 0 || p2 >= L) continue;
-    const int f2 = (p2 + 1) / B * B;
-    if (f2 == p2 + 1) continue;
-    const uint16_t* col = K + (ko[seq] + f2) * kD + dim;
-    float s = 0.f;
-    for (int key = f2; key <= p2; ++key) s += bf16_bits_to_float(col[(int64_t)(key - f2) * kD]);
-    part[qi * kD + dim] = s / (float)(p2 + 1 - f2);
+  const int64_t slots = nsplit_max + 1;  // stored sums per group
+  if (kMode == kPartial) {
+    partial[((int64_t)g * slots + y) * kRouteThreads + tid] = acc;
+    return;
   }
-  __syncthreads();
-  if (valid && nfull * B != n) {
-    const float4* row = reinterpret_cast<const float4*>(part + qq * kD);
-    float d = 0.f;
-#pragma unroll
-    for (int i = 0; i < kD / 4; ++i) {
-      const float4 a = row[i];
-      d = fmaf(qreg[4 * i + 0], a.x, d);
-      d = fmaf(qreg[4 * i + 1], a.y, d);
-      d = fmaf(qreg[4 * i + 2], a.z, d);
-      d = fmaf(qreg[4 * i + 3], a.w, d);
-    }
-    acc += fmaxf(d, 0.f);
+  if (kMode == kFinish && valid) {
+    const float* pp = partial + (int64_t)g * slots * kRouteThreads + tid;
+    for (int j = 0; j <= ns; ++j) acc += pp[(int64_t)j * kRouteThreads];
   }
 
   float r = -INFINITY;
@@ -173,19 +236,56 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
 int route_group_size(int H) { return H >= kRouteThreads ? 1 : kRouteThreads / H; }
 
+// Most ranges of pooled blocks per group (the device takes fewer when there
+// are more groups): split only when the groups alone leave SMs idle, into
+// ranges of about 16 blocks or more.
+int route_split_count(const misa_problem_t& p, int max_groups, int sms) {
+  if (max_groups <= 0 || max_groups >= sms) return 1;
+  const int max_blocks = (int)(p.max_seq_len / p.block);
+  const int by_work = (max_blocks + 15) / 16;
+  const int n = by_work < sms ? by_work : sms;
+  return n < 2 ? 1 : n;
+}
+
+size_t route_split_bytes(int max_groups, int nsplit) {
+  return nsplit <= 1 ? 0 : (size_t)max_groups * (nsplit + 1) * kRouteThreads * sizeof(float);
+}
+
 int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, const uint16_t* K,
                  const float* Kbar, int m, int32_t* heads, uint16_t* q_r, float* w_r,
                  float* router_scores, const int4* groups, const int* group_count,
-                 int max_groups, int G, cudaStream_t st) {
+                 int max_groups, int G, int nsplit, float* partial, cudaStream_t st) {
   if (max_groups <= 0) return MISA_OK;
   const int smem = (kChunk * kD + G * kD + G * p.num_heads) * (int)sizeof(float);
-  int rc = set_smem_limit((const void*)route_kernel, smem);
-  if (rc) return rc;
-  ProfScope ps("route", st);
-  route_kernel<<<max_groups, kRouteThreads, smem, st>>>(
+  const int sms = num_sms();
+  int rc;
+  if (nsplit <= 1 || !partial) {
+    if ((rc = set_smem_limit((const void*)route_kernel<kWhole>, smem))) return rc;
+    ProfScope ps("route", st);
+    route_kernel<kWhole><<<max_groups, kRouteThreads, smem, st>>>(
+        q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
+        p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), 1, sms,
+        nullptr);
+    return cuda_fail(cudaGetLastError(), "route_kernel");
+  }
+  if ((rc = set_smem_limit((const void*)route_kernel<kPartial>, smem))) return rc;
+  if ((rc = set_smem_limit((const void*)route_kernel<kFinish>, smem))) return rc;
+  {
+    // One CTA per (group, range) and one per group for its partial block;
+    // the device uses the first count * (ns + 1) of them.
+    ProfScope ps("route", st);
+    route_kernel<kPartial><<<max_groups * (nsplit + 1), kRouteThreads, smem, st>>>(
+        q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
+        p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), nsplit, sms,
+        partial);
+    if ((rc = cuda_fail(cudaGetLastError(), "route_kernel (ranges)"))) return rc;
+  }
+  ProfScope ps("route_finish", st);
+  route_kernel<kFinish><<<max_groups, kRouteThreads, smem, st>>>(
       q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
-      p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr());
-  return cuda_fail(cudaGetLastError(), "route_kernel");
+      p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), nsplit, sms,
+      partial);
+  return cuda_fail(cudaGetLastError(), "route_kernel (finish)");
 }
 
 }  // namespace misa

@@ -351,9 +351,20 @@ int launch_score(const ScoreArgs& a, cudaStream_t st) {
   if (rc) return rc;
   rc = make_kmajor_map(&qmap, a.qsel, (int64_t)a.p->num_queries * a.m, 32);
   if (rc) return rc;
-  const int64_t work = (int64_t)a.max_groups * a.max_tiles;
-  int tps = (int)((work + 8 * kSms - 1) / (8 * kSms));
-  tps = max(1, min(tps, 64));
+  // Prefill-sized problems: about 8 CTAs per SM over the whole causal work,
+  // for balance.  Decode-sized problems (fewer groups than SMs): one wave, so
+  // that each CTA streams a long key range through its pipeline rather than
+  // paying its set-up for a few tiles in many waves.
+  const int sms = num_sms();
+  int tps;
+  if (a.max_groups < sms) {
+    const int splits = max(1, sms / a.max_groups);
+    tps = (a.max_tiles + splits - 1) / splits;
+  } else {
+    const int64_t work = (int64_t)a.max_groups * a.max_tiles;
+    tps = (int)((work + 8 * sms - 1) / (8 * sms));
+    tps = max(1, min(tps, 64));
+  }
   const int splits = (a.max_tiles + tps - 1) / tps;
   if (splits > 65535) {
     set_error("score: %d key splits exceed the grid limit", splits);

@@ -13,6 +13,14 @@
 // k-th element is consumed exactly, which in practice happens after the
 // first two score digits.  A last pass writes every element whose key prefix
 // is at or above the threshold prefix: exactly min(k, n) of them.
+//
+// Decode batches have few rows, each a long prefix.  There a row is split
+// over a thread-block cluster: each CTA loads its slice of the row once into
+// shared memory as 64-bit keys, builds its digit histogram there, and reads
+// the other CTAs' histograms over distributed shared memory; every CTA then
+// holds the same row histogram and takes the same decision, so the passes
+// need no further exchange.  The output slots come from one counter in the
+// first CTA of the cluster.
 #include "common.cuh"
 #include "internal.h"
 
@@ -168,12 +176,248 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- cluster form
+constexpr int kClusterCap = 16384;  // keys per CTA held in shared memory
+constexpr int kMaxCluster = 8;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA of the cluster; orders shared-memory writes
+// before the barrier against reads after it, cluster-wide.
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t addr, uint32_t x) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(x)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t* warp_tot) {
+  const uint32_t off = block_exclusive_scan(x, warp_tot);
+  __shared__ uint32_t total;
+  if (threadIdx.x == kTopkThreads - 1) total = off + x;
+  __syncthreads();
+  const uint32_t r = total;
+  __syncthreads();
+  return r;
+}
+
+// Grid: rows x C CTAs, cluster (C,1,1); C = gridDim.x / rows.
+__global__ void __launch_bounds__(kTopkThreads, 1)
+    topk_cluster_kernel(const float* __restrict__ I, int64_t ld, const int32_t* __restrict__ tok,
+                        int n_fixed, const int64_t* __restrict__ ko,
+                        const int32_t* __restrict__ qo, const int32_t* __restrict__ q_pos, int S,
+                        int q_lo, int k, int C, int32_t* __restrict__ idx_out,
+                        float* __restrict__ val_out, uint32_t* status) {
+  extern __shared__ __align__(16) uint64_t keys[];  // [kClusterCap]; 0 = not a candidate
+  __shared__ uint32_t hist[2][kMaxBins];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_valid, s_out;
+  __shared__ uint32_t sel_bin, sel_above, sel_count;
+
+  const uint32_t rank = cluster_ctarank();
+  const int row = blockIdx.x / C;
+  const int t = q_lo + row;
+  const int s = upper_segment<int32_t>(qo, S, t);
+  const int64_t L = ko[s + 1] - ko[s];
+  int pos = q_pos[t];
+  if (pos < 0 || pos >= L) pos = -1;
+
+  Row r;
+  r.I = I + (int64_t)row * ld;
+  r.tok = tok ? tok + (int64_t)t * n_fixed : nullptr;
+  r.n = tok ? n_fixed : pos + 1;
+  r.pos = pos;
+  int32_t* idx = idx_out + (int64_t)t * k;
+  float* val = val_out + (int64_t)t * k;
+
+  const int chunk = (((r.n + C - 1) / C) + 3) & ~3;
+  if (chunk > kClusterCap) {  // uniform over the cluster: no CTA reaches a barrier
+    if (rank == 0 && threadIdx.x == 0) set_status(status, MISA_STATUS_BOUNDS);
+    return;
+  }
+  const int e0 = (int)rank * chunk;
+  const int nloc = max(0, min(r.n, e0 + chunk) - e0);
+
+  // Load the slice with 8 independent loads in flight per thread.
+  uint32_t local_valid = 0;
+  constexpr int kU = 8;
+  for (int i0 = 0; i0 < nloc; i0 += kU * kTopkThreads) {
+    float v[kU];
+    int tk[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * kTopkThreads + threadIdx.x;
+      v[u] = 0.f;
+      tk[u] = -1;
+      if (i < nloc) {
+        v[u] = r.I[e0 + i];
+        tk[u] = r.tok ? r.tok[e0 + i] : e0 + i;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * kTopkThreads + threadIdx.x;
+      if (i >= nloc) continue;
+      const bool ok = tk[u] >= 0 && (!r.tok || tk[u] <= r.pos);
+      // A real key is never 0: its low word is 0xFFFFFFFF - token >= 2^31.
+      keys[i] = ok ? (static_cast<uint64_t>(order_key(v[u])) << 32) |
+                         static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(tk[u]))
+                   : 0ull;
+      local_valid += ok;
+    }
+  }
+  const uint32_t cta_valid = block_sum(local_valid, warp_tot);
+  if (threadIdx.x == 0) {
+    s_valid = cta_valid;
+    s_out = 0;
+  }
+  cluster_barrier();  // s_valid of every CTA and s_out of CTA 0 are set
+  uint32_t n_valid = 0;
+  for (int q = 0; q < C; ++q) n_valid += dsmem_ld(dsmem_addr(&s_valid, q));
+
+  constexpr int kShift[6] = {53, 42, 32, 21, 10, 0};
+  constexpr int kWidth[6] = {11, 11, 10, 11, 11, 10};
+  uint64_t prefix = 0;
+  uint32_t remaining = (uint32_t)k;
+  int shift = 64;
+  bool done = n_valid <= (uint32_t)k;
+
+  for (int p = 0; p < 6 && !done; ++p) {
+    const int width = kWidth[p], sh = kShift[p];
+    const int nb = 1 << width;
+    const uint32_t mask = (uint32_t)nb - 1u;
+    uint32_t* h = hist[p & 1];
+    // hist[p & 1] was last read remotely in pass p-2, before every CTA
+    // arrived at pass p-1's cluster barrier: safe to clear.
+    for (int b = threadIdx.x; b < nb; b += kTopkThreads) h[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nloc; i += kTopkThreads) {
+      const uint64_t key = keys[i];
+      if (key == 0ull) continue;
+      if (p == 0 || (key >> (sh + width)) == prefix) atomicAdd(&h[(uint32_t)(key >> sh) & mask], 1u);
+    }
+    cluster_barrier();  // every CTA's histogram of this pass is complete
+    const int bpt = nb / kTopkThreads;  // 1 or 2
+    uint32_t c[2] = {0, 0};
+    for (int j = 0; j < bpt; ++j) {
+      const int bin = nb - 1 - (threadIdx.x * bpt + j);
+      for (int q = 0; q < C; ++q) c[j] += dsmem_ld(dsmem_addr(h + bin, q));
+    }
+    const uint32_t above0 = block_exclusive_scan(c[0] + c[1], warp_tot);
+    uint32_t above = above0;
+    for (int j = 0; j < bpt; ++j) {
+      if (above < remaining && above + c[j] >= remaining) {
+        sel_bin = (uint32_t)(nb - 1 - (threadIdx.x * bpt + j));
+        sel_above = above;
+        sel_count = c[j];
+      }
+      above += c[j];
+    }
+    __syncthreads();
+    remaining -= sel_above;
+    prefix = (prefix << width) | sel_bin;
+    shift = sh;
+    if (sel_count == remaining) done = true;
+    __syncthreads();
+  }
+
+  // Output: this CTA's selected keys, at slots reserved from CTA 0's counter.
+  uint32_t mine = 0;
+  for (int i = threadIdx.x; i < nloc; i += kTopkThreads) {
+    const uint64_t key = keys[i];
+    mine += key != 0ull && (shift == 64 || (key >> shift) >= prefix);
+  }
+  const uint32_t off = block_exclusive_scan(mine, warp_tot);
+  __shared__ uint32_t base;
+  if (threadIdx.x == kTopkThreads - 1) base = dsmem_atomic_add(dsmem_addr(&s_out, 0), off + mine);
+  __syncthreads();
+  uint32_t slot = base + off;
+  for (int i = threadIdx.x; i < nloc; i += kTopkThreads) {
+    const uint64_t key = keys[i];
+    if (key == 0ull || !(shift == 64 || (key >> shift) >= prefix)) continue;
+    if (slot < (uint32_t)k) {
+      idx[slot] = (int)(0xFFFFFFFFu - (uint32_t)key);
+      val[slot] = key_to_float((uint32_t)(key >> 32));
+    } else {
+      set_status(status, MISA_STATUS_BOUNDS);  // duplicate tokens in a candidate row
+    }
+    ++slot;
+  }
+  if (rank == 0) {
+    const int filled = n_valid < (uint32_t)k ? (int)n_valid : k;
+    for (int j = filled + threadIdx.x; j < k; j += kTopkThreads) {
+      idx[j] = -1;
+      val[j] = -INFINITY;
+    }
+  }
+  cluster_barrier();  // CTA 0's counter stays alive until every CTA has used it
+}
+
 }  // namespace
+
+// Cluster size for a top-k over `rows` rows of at most nmax elements: a power
+// of two large enough to hold a row slice in shared memory, grown while all
+// rows still fit one wave of CTAs; 1 = the one-CTA-per-row kernel.
+int topk_cluster_size(int rows, int64_t nmax, int sms) {
+  if (rows <= 0 || rows * 2 > sms || nmax < 4096) return 1;
+  const int64_t need = (nmax + kClusterCap - 1) / kClusterCap;
+  int c = 1;
+  while (c < need) c <<= 1;
+  while (c * 2 <= kMaxCluster && rows * c * 2 <= sms) c <<= 1;  // stay within one wave
+  if (c > kMaxCluster || (int64_t)c * kClusterCap < nmax) return 1;
+  return c;
+}
 
 int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32_t* tok,
                 int n_fixed, int q_lo, int q_hi, int k, int32_t* idx, float* val,
                 cudaStream_t st) {
   if (q_hi <= q_lo) return MISA_OK;
+  const int rows = q_hi - q_lo;
+  const int64_t nmax = tok ? n_fixed : p.max_seq_len;
+  const int C = topk_cluster_size(rows, nmax, num_sms());
+  if (C > 1) {
+    const int smem = kClusterCap * (int)sizeof(uint64_t);
+    int rc = set_smem_limit((const void*)topk_cluster_kernel, smem);
+    if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * C));
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfScope ps("topk", st);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, I, ld, tok, n_fixed,
+                                       p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo,
+                                       k, C, idx, val, status_ptr());
+    return cuda_fail(e, "topk_cluster_kernel");
+  }
   ProfScope ps("topk", st);
   topk_kernel<<<q_hi - q_lo, kTopkThreads, 0, st>>>(I, ld, tok, n_fixed, p.key_offsets,
                                                     p.query_offsets, p.q_pos, p.num_seqs, q_lo,
