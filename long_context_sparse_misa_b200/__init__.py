@@ -4,7 +4,7 @@ Argument marshalling only: every step of the indexer runs in the CUDA
 kernels behind the C ABI declared in include/misa.h.  PyTorch provides
 device memory and streams.  There is no CPU fallback: importing this package
 without a built libmisa.so raises ImportError (build it with
-``python -m long_context_sparse_misa_b200.build``).
+``python long_context_sparse_misa_b200/build.py``).
 
 Method: "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
 Inference" -- a block-pooled router keeps m of the H indexer heads per query,
@@ -34,7 +34,7 @@ EXPORTED = (
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m long_context_sparse_misa_b200.build` (needs nvcc)")
+                      "`python long_context_sparse_misa_b200/build.py` (needs nvcc)")
 lib = ctypes.CDLL(LIB_PATH)
 
 _c_i32, _c_i64, _c_sz, _c_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p

@@ -1,6 +1,6 @@
 """Build libmisa.so (sm_100a) in-tree with nvcc.
 
-    python -m long_context_sparse_misa_b200.build [--force] [--verbose]
+    python long_context_sparse_misa_b200/build.py [--force] [--verbose]
 
 Each .cu under csrc/ is compiled to an object in _build/ (parallel), then
 linked into long_context_sparse_misa_b200/libmisa.so with the CUDA runtime

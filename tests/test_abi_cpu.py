@@ -11,8 +11,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def misa():
-    from long_context_sparse_misa_b200 import build
-    build.build()
+    # The build script is loaded by path: importing the package needs the library.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_misa_build", os.path.join(ROOT, "long_context_sparse_misa_b200", "build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()
     import long_context_sparse_misa_b200 as m
     return m
 
