@@ -118,6 +118,24 @@ int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const
                const float* Kbar, int32_t m, int32_t* heads, uint16_t* q_r, float* w_r,
                float* router_scores, void* ws, size_t ws_bytes, misa_stream_t stream);
 
+/* misa_route without a caller workspace: its scratch is a fixed 4 MiB device
+ * array inside the library (one per device), for callers that cannot
+ * allocate on the decode path (a host runtime with no device allocator of
+ * its own, or code that must not call cudaMalloc there).  No counterpart in
+ * the paper.  Arguments and results as misa_route, which it runs with that
+ * array as its workspace; it allocates no memory.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's address; make it before capturing a stream that uses the call.
+ *   - Nothing in the array needs to start at zero.
+ *   - Calls on one device must not overlap in execution: they share the
+ *     array and race on it.  Issue them on one stream, or order them.
+ *   - MISA_ERR_UNSUPPORTED when the problem needs more than 4 MiB of router
+ *     scratch (the message gives both sizes); MISA_ERR_INVALID_ARG while
+ *     tracing is on for the calling thread. */
+int misa_route_static(const misa_problem_t* p, const uint16_t* q, const float* w,
+                      const uint16_t* K, const float* Kbar, int32_t m, int32_t* heads,
+                      uint16_t* q_r, float* w_r, float* router_scores, misa_stream_t stream);
+
 /* Steps 3+4 -- routed token scoring and per-query top-k (same section,
  * Sparse Token Scoring: only the routed heads score the full prefix; the
  * top-k tokens come from these reduced scores).

@@ -19,7 +19,7 @@ import os
 __all__ = [
     "LIB_PATH", "lib", "MisaError", "Problem", "workspace_size", "block_offsets", "pool_keys",
     "route", "score_topk", "hier_rerank", "dsa_index_dense", "stream_status",
-    "selftest_timeout", "EXPORTED", "Indexer", "profile_enable", "profile_collect",
+    "selftest_timeout", "route_static", "EXPORTED", "Indexer", "profile_enable", "profile_collect",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmisa.so")
@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmisa.so"
 # Every symbol include/misa.h declares.
 EXPORTED = (
     "misa_workspace_size", "misa_block_offsets", "misa_pool_keys", "misa_route",
-    "misa_score_topk", "misa_hier_rerank", "dsa_index_dense", "misa_stream_status",
+    "misa_route_static", "misa_score_topk", "misa_hier_rerank", "dsa_index_dense", "misa_stream_status",
     "misa_selftest_timeout", "misa_profile_enable", "misa_profile_collect",
     "misa_last_error_string",
 )
@@ -57,6 +57,8 @@ _sig = {
     "misa_pool_keys": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p]),
     "misa_route": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p,
                                   _c_p, _c_sz, _c_p]),
+    "misa_route_static": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p,
+                                         _c_p, _c_p]),
     "misa_score_topk": (ctypes.c_int, [_PP, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p,
                                        _c_i64, _c_p, _c_sz, _c_p]),
     "misa_hier_rerank": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p,
@@ -173,6 +175,13 @@ def route(prob: Problem, q, w, K, Kbar, m: int, heads, q_r, w_r, router_scores, 
     _check(lib.misa_route(prob.ref, _ptr(q), _ptr(w), _ptr(K), _ptr(Kbar), m, _ptr(heads),
                           _ptr(q_r), _ptr(w_r), _ptr(router_scores), _ptr(ws), ws.numel(),
                           _stream(stream)), "misa_route")
+
+
+def route_static(prob: Problem, q, w, K, Kbar, m: int, heads, q_r, w_r, router_scores,
+                 stream=None) -> None:
+    _check(lib.misa_route_static(prob.ref, _ptr(q), _ptr(w), _ptr(K), _ptr(Kbar), m,
+                                 _ptr(heads), _ptr(q_r), _ptr(w_r), _ptr(router_scores),
+                                 _stream(stream)), "misa_route_static")
 
 
 def score_topk(prob: Problem, q_r, w_r, m: int, K, k: int, idx, val, ws, scores_dbg=None,

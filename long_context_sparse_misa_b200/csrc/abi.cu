@@ -350,6 +350,16 @@ __global__ void selftest_timeout_kernel(long long wait_ns, uint32_t* status) {
 }
 
 }  // namespace
+// Workspace that misa_route uses for this problem on its fastest path (the
+// tensor-core router where it applies, else the CUDA-core router with its
+// pooled-block ranges).  The problem must have passed check_problem.
+size_t route_path_bytes(const misa_problem_t* p) {
+  return route_tc_applies(p) ? route_tc_bytes(p) : route_bytes(p);
+}
+
+// Whether tracing is on for the calling host thread.
+bool tracing_enabled() { return t_prof_on; }
+
 }  // namespace misa
 
 using namespace misa;

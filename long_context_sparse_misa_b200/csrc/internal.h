@@ -31,6 +31,10 @@ int make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int box_ro
 int set_smem_limit(const void* kernel, int bytes);
 // SMs of the current device.
 int num_sms();
+// Workspace misa_route uses on its fastest path for a checked problem.
+size_t route_path_bytes(const misa_problem_t* p);
+// Whether tracing (misa_profile_enable) is on for the calling host thread.
+bool tracing_enabled();
 
 // Tracing: brackets one kernel launch with events on `st` when profiling is on.
 struct ProfScope {
