@@ -16,11 +16,12 @@
 // tiles of K stream through a 4-stage TMA ring (A operand); tcgen05.mma
 // accumulates 128 keys x 256 columns in TMEM, two buffers.
 //
-// Epilogue (8 warps: TMEM lane quarter = warp % 4, column half = which of
-// the two warps of that quarter), per tile: two tcgen05.ld of 32 columns
-// before each wait, the TMEM buffer released after the second pair, then per
-// key and query I = sum_j w_j ReLU(acc_j), the causal mask, and the
-// streaming selection:
+// Epilogue (16 warps, four per SM sub-partition so that their dependency
+// chains overlap: TMEM lane quarter = warp % 4, column quarter = which of the
+// four warps of that lane quarter, i.e. 64 columns = 64/m queries each), per
+// tile: tcgen05.ld of 32 columns, wait, then per key and query
+// I = sum_j w_j ReLU(acc_j) (the TMEM buffer is released after the warp's
+// last load), the causal mask, and the streaming selection:
 //   * probe: a group first scores every 8th tile of its prefix and keeps a
 //     128-bin histogram per query (1/8-octave bins of the order-preserving
 //     score key, anchored 14 octaves below the first scored tile's maximum).
@@ -45,12 +46,15 @@
 namespace misa {
 namespace {
 
-constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
-constexpr int kEpiWarps = 8;
 constexpr int kStages = 4;
 constexpr int kStageBytes = kTileKeys * kD * 2;  // 32 KB
 constexpr int kHalfBytes = kStageBytes / 2;
 constexpr int kN = 256;                          // MMA N = group columns
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;       // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
+constexpr int kParts = kEpiWarps / 4;            // column parts per TMEM lane quarter
+constexpr int kColsPerWarp = kN / kParts;
 constexpr int kQHalfBytes = kN * 128;            // 32 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kTmemCols = 2 * kN;
@@ -63,10 +67,12 @@ constexpr int kProbeStride = 8;                  // probe every 8th tile ...
 constexpr int kProbeOff = 4;                     // ... starting at tile 4
 constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
 
+// The per-warp select scratch of the final selection reuses the probe
+// histograms (free by then).
+static_assert(kEpiWarps * kSelBins <= kMaxG * kBins, "select scratch must fit the histograms");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
                            kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ + kMaxG * 4 * 4 /*wc*/ +
-                           kMaxG * kBins * 4 /*hist*/ + kEpiWarps * kSelBins * 4 /*select*/ +
-                           32 * 8 /*barriers*/ + 16;
+                           kMaxG * kBins * 4 /*hist, select*/ + 32 * 8 /*barriers*/ + 16;
 
 struct Smem {
   uint8_t* q;
@@ -79,7 +85,7 @@ struct Smem {
   int* base;  // histogram anchor per query
   int* wc;    // [kMaxG][4] sub-buffer counts
   uint32_t* hist;
-  uint32_t* sel;
+  uint32_t* sel;  // aliases hist
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -106,8 +112,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
   s.wc = s.base + kMaxG;
   s.hist = reinterpret_cast<uint32_t*>(s.wc + kMaxG * 4);
-  s.sel = s.hist + kMaxG * kBins;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.sel + kEpiWarps * kSelBins);
+  s.sel = s.hist;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.hist + kMaxG * kBins);
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
@@ -258,7 +264,7 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* cnt, int 
     // Pass 1: entries above the threshold bin go out; threshold-bin entries
     // are compacted to the front of the region.  Each lane issues kU loads
     // before using any of them (the buffer is mostly beyond L2).
-    constexpr int kU = 32;
+    constexpr int kU = 16;
     int zpos = 0;
     for (int r = 0; r < 4; ++r) {
       const uint2* sb = region + r * subcap;
@@ -365,16 +371,16 @@ __device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
 }
 
 template <int MH>
-__global__ void __launch_bounds__(kThreads, 1)
+// 18 warps at 96 registers each: one CTA per SM.
+__global__ void __maxnreg__(96)
     score_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap qmap, const float* __restrict__ wsel,
                         const int64_t* __restrict__ ko, Sched sc, int k, uint2* __restrict__ cand,
                         int64_t subcap, int32_t* __restrict__ idx_out,
                         float* __restrict__ val_out, uint32_t* status) {
   constexpr int G = kN / MH;          // queries per group
-  constexpr int QH = G / 2;           // queries per column half
-  constexpr int QPW = QH / 2;         // queries per 64-column window
-  static_assert(MH >= 8 && MH <= 64 && G <= kMaxG && QPW >= 1, "unsupported head count");
+  constexpr int QH = G / kParts;      // queries per epilogue warp (its column part)
+  static_assert(MH >= 8 && MH <= 64 && G <= kMaxG && QH >= 1, "unsupported head count");
   extern __shared__ uint8_t smem_raw[];
 
   const int count = *sc.count;
@@ -484,11 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;                  // 0..7
+    const int e = warp - 2;                  // 0..kEpiWarps-1
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
-    const int half = e >> 2;                 // column half: queries half*QH .. half*QH+QH-1
+    const int half = e >> 2;                 // column part: queries half*QH .. half*QH+QH-1
     const int lrow = quarter * 32 + lane;    // key row of the tile
-    const int et = threadIdx.x - 64;         // 0..255
+    const int et = threadIdx.x - 64;         // 0..kEpiThreads-1
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t ephase = 0;
@@ -502,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int np = probe_tiles(probe, ntiles);
       const int64_t L = ko[seq + 1] - ko[seq];
       // Group state: column weights, query limits, selection state.
-      {
+      if (et < kN) {
         const int qi = et / MH;
         s.w[et] = qi < nq ? wsel[(int64_t)(qb + qi) * MH + (et - qi * MH)] : 0.f;
       }
@@ -517,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         s.tau[et] = p >= 0 ? -INFINITY : INFINITY;  // padding / invalid slots never append
         s.maxkey[et] = 0u;
       }
-      for (int i = et; i < G * kBins; i += 256) s.hist[i] = 0u;
+      for (int i = et; i < G * kBins; i += kEpiThreads) s.hist[i] = 0u;
       // This warp's slot counters (one per query; only this warp touches
       // them) and its sub-buffer of its first query; query stride 4 * subcap.
       int* mycnt = s.wc + quarter * kMaxG + half * QH;  // [quarter][query]
@@ -538,30 +544,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = tb & 1;
         if (!(ok = warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status))) break;
         tc_fence_after();
-        const uint32_t taddr = lane_addr + buf * kN + half * 128;
+        const uint32_t taddr = lane_addr + buf * kN + half * kColsPerWarp;
         float sc_[QH];
+        if constexpr (MH <= 32) {
+          // One 32-column load at a time: 32/MH whole queries per load.
+          constexpr int QPL = 32 / MH;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+          for (int hh = 0; hh < kColsPerWarp / 32; ++hh) {
+            float v[32];
+            tmem_ld32(taddr + hh * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+            if (hh == kColsPerWarp / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&s.tempty[buf]);
+            }
+#pragma unroll
+            for (int q2 = 0; q2 < QPL; ++q2)
+              sc_[hh * QPL + q2] = relu_wsum<MH>([&](int j) { return v[q2 * MH + j]; },
+                                                 s.w + half * kColsPerWarp + hh * 32 + q2 * MH);
+          }
+        } else {
+          // MH == 64: the warp's one query spans both 32-column loads.
+          static_assert(MH != 64 || (QH == 1 && kColsPerWarp == 64), "one query per warp");
           float v[2][32];
-          tmem_ld32(taddr + (2 * hh) * 32, v[0]);
-          tmem_ld32(taddr + (2 * hh + 1) * 32, v[1]);
+          tmem_ld32(taddr, v[0]);
+          tmem_ld32(taddr + 32, v[1]);
           tmem_wait_ld();
           reg_fence32(v[0]);
           reg_fence32(v[1]);
-          if (hh == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.tempty[buf]);
-          }
-#pragma unroll
-          for (int q2 = 0; q2 < QPW; ++q2) {
-            sc_[hh * QPW + q2] = relu_wsum<MH>(
-                [&](int j) {
-                  const int col = q2 * MH + j;
-                  return v[col >> 5][col & 31];
-                },
-                s.w + half * 128 + hh * 64 + q2 * MH);
-          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[buf]);
+          sc_[0] = relu_wsum<MH>([&](int j) { return v[j >> 5][j & 31]; }, s.w + half * kColsPerWarp);
         }
         const int key = tile * kTileKeys + lrow;
         if (step == 0) {
