@@ -279,17 +279,25 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, 
 // summation order every scoring kernel uses (so all paths agree bit for bit):
 // even heads into a0, odd heads into a1 (one packed FMA per pair), then
 // a0 + a1.  `col(j)` gives the accumulator value of head j, `wq` the head
-// weights.
+// weights as stored by relu_weight (halved).  ReLU is formed as
+// a + |a| = 2 max(a, 0), exactly, on the FMA pipe (the |a| is an operand
+// modifier) rather than as max(a, 0) on the integer/logic pipe; with the
+// halved weight each product (w/2)(2 max(a, 0)) equals w max(a, 0) exactly,
+// so the sum is the same as with the plain form.
+__device__ __forceinline__ float relu_weight(float w) { return 0.5f * w; }
+
 template <int MH, typename ColFn>
 __device__ __forceinline__ float relu_wsum(ColFn col, const float* wq) {
   float a0 = 0.f, a1 = 0.f;
   if constexpr (MH == 1) {
-    a0 = fmaf(wq[0], fmaxf(col(0), 0.f), a0);
+    const float c0 = col(0);
+    a0 = fmaf(wq[0], c0 + fabsf(c0), a0);
   } else {
 #pragma unroll
     for (int j = 0; j < MH; j += 2) {
       const float2 wj = *reinterpret_cast<const float2*>(wq + j);
-      ffma2(a0, a1, wj.x, wj.y, fmaxf(col(j), 0.f), fmaxf(col(j + 1), 0.f));
+      const float c0 = col(j), c1 = col(j + 1);
+      ffma2(a0, a1, wj.x, wj.y, c0 + fabsf(c0), c1 + fabsf(c1));
     }
   }
   return a0 + a1;

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Per-column head weight and per-query causal limit / output row.
     for (int c = threadIdx.x - 64; c < kMaxN; c += 128) {
       const int qi = c / MH;
-      s.w[c] = (c < nq * MH) ? wsel[(int64_t)(qb + qi) * MH + (c - qi * MH)] : 0.f;
+      s.w[c] = (c < nq * MH) ? relu_weight(wsel[(int64_t)(qb + qi) * MH + (c - qi * MH)]) : 0.f;
     }
     for (int qi = threadIdx.x - 64; qi < kMaxN; qi += 128) {
       int pos = -1;

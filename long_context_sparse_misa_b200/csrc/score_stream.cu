@@ -510,7 +510,7 @@ __global__ void __maxnreg__(96)
       // Group state: column weights, query limits, selection state.
       if (et < kN) {
         const int qi = et / MH;
-        s.w[et] = qi < nq ? wsel[(int64_t)(qb + qi) * MH + (et - qi * MH)] : 0.f;
+        s.w[et] = qi < nq ? relu_weight(wsel[(int64_t)(qb + qi) * MH + (et - qi * MH)]) : 0.f;
       }
       if (et < G) {
         int p = -1;
