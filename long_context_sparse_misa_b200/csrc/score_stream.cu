@@ -32,8 +32,9 @@
 //   * main pass over all tiles: a key is appended to query q's candidates
 //     only if I >= tau_q.  Each (query, lane quarter) has a private
 //     sub-buffer with one slot per key the quarter can see, so nothing can
-//     overflow; slot ranks come from per-query ballots, and each lane issues
-//     its appends in rounds (as many rounds as the busiest lane has appends).
+//     overflow; per query, a ballot ranks the passing lanes and one
+//     predicated store writes them contiguously after the query's earlier
+//     appends (the running count is kept, warp-uniform, in registers).
 //   * check and select: every key scoring at least tau_q was appended, so if
 //     at least min(k, n) keys were appended the exact top-k is among them.
 //     The owner warp then histograms the candidates, takes those above the
@@ -138,23 +139,7 @@ __device__ __forceinline__ int score_bin(uint32_t key, int base) {
   return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
 }
 
-// a[q] for a per-lane q without dynamic register indexing: a select tree
-// over the bits of q.
-template <int N>
-__device__ __forceinline__ float pick(const float (&a)[N], int q) {
-  static_assert((N & (N - 1)) == 0, "power of two");
-  float t[N];
-#pragma unroll
-  for (int i = 0; i < N; ++i) t[i] = a[i];
-#pragma unroll
-  for (int w = N / 2, bit = 0; w >= 1; w /= 2, ++bit) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = ((q >> bit) & 1) ? t[2 * i + 1] : t[2 * i];
-  }
-  return t[0];
-}
-
-// Barrier over the 8 epilogue warps (bounded; warp-uniform result).
+// Barrier over the epilogue warps (bounded; warp-uniform result).
 __device__ __forceinline__ bool ep_barrier(Smem& s, uint32_t& phase, uint32_t* status) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(s.ebar);
@@ -527,7 +512,9 @@ __global__ void __maxnreg__(96)
       // This warp's slot counters (one per query; only this warp touches
       // them) and its sub-buffer of its first query; query stride 4 * subcap.
       int* mycnt = s.wc + quarter * kMaxG + half * QH;  // [quarter][query]
-      if (lane < QH) mycnt[lane] = 0;
+      int cnt[QH];  // appends so far per query (warp-uniform)
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
       uint2* mysub = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 4 * subcap +
                      (int64_t)quarter * subcap;
       const int qstride = 4 * static_cast<int>(subcap);
@@ -641,36 +628,26 @@ __global__ void __maxnreg__(96)
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
         }
-        // Streaming selection.  Each lane learns which of the warp's QH
-        // queries it appends to (a bit mask); the ballot, slot counter and
-        // histogram anchor of query qq live on lane qq and are fetched by
-        // shuffle.  The warp then issues one store and one histogram
-        // reduction per round, and there are as many rounds as the busiest
-        // lane has appends (usually a few), not QH.
-        uint32_t mymask = 0, balJ = 0;
-        // tiles wholly below every query's position need no causal compare
+        // Streaming selection: per query one ballot gives each passing lane
+        // its slot after the query's earlier appends (the count is the same
+        // in every lane of the warp), then one predicated 8-byte store per
+        // query writes the warp's appends contiguously.
+        // Tiles wholly below every query's position need no causal compare.
         const bool full_tile = (tile + 1) * kTileKeys <= minpos + 1;
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
           const bool take = (full_tile || key <= s.pos[half * QH + qq]) && sc_[qq] >= tauR[qq];
           const uint32_t bq = __ballot_sync(0xffffffffu, take);
-          mymask |= (take ? 1u : 0u) << qq;
-          balJ = lane == qq ? bq : balJ;
+          st_global_u2_if(mysub + (int64_t)qq * qstride + cnt[qq] + __popc(bq & lt),
+                          __float_as_uint(sc_[qq]), static_cast<uint32_t>(key), take);
+          cnt[qq] += __popc(bq);
         }
-        int c0J = lane < QH ? mycnt[lane] : 0;
-        while (__any_sync(0xffffffffu, mymask != 0)) {
-          const bool act = mymask != 0;
-          const int q = act ? __ffs(mymask) - 1 : 0;
-          mymask &= mymask - 1u;
-          const uint32_t bq = __shfl_sync(0xffffffffu, balJ, q);
-          const int cq = __shfl_sync(0xffffffffu, c0J, q);
-          const float v = pick<QH>(sc_, q);
-          st_global_u2_if(mysub + q * qstride + cq + __popc(bq & lt), __float_as_uint(v),
-                          static_cast<uint32_t>(key), act);
-        }
-        if (lane < QH) mycnt[lane] = c0J + __popc(balJ);
       }
       if (!ok) break;
+      if (lane == 0) {
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) mycnt[qq] = cnt[qq];
+      }
       if (!(ok = ep_barrier(s, ephase, status))) break;
       for (int qi = e; qi < nq; qi += kEpiWarps) {
         const int t = s.row[qi];
