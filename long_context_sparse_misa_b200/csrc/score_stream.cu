@@ -139,6 +139,28 @@ __device__ __forceinline__ int score_bin(uint32_t key, int base) {
   return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
 }
 
+// Columns C*16 .. C*16+15 of a warp's 64: the head-weighted ReLU sums in the
+// order of relu_wsum (even heads into a0, odd into a1, then a0 + a1), with
+// a query's running sums carried across chunks when it spans several.
+template <int MH, int C, int QH>
+__device__ __forceinline__ void chunk_wsum(const float (&v)[16], const float* wcol, float& a0,
+                                           float& a1, float (&sc)[QH]) {
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    constexpr int kBase = C * 16;
+    const int col = kBase + 2 * p;
+    const int j = col % MH;
+    if (j == 0) {
+      a0 = 0.f;
+      a1 = 0.f;
+    }
+    const float2 wj = *reinterpret_cast<const float2*>(wcol + col);
+    const float c0 = v[2 * p], c1 = v[2 * p + 1];
+    ffma2(a0, a1, wj.x, wj.y, c0 + fabsf(c0), c1 + fabsf(c1));
+    if (j + 2 == MH) sc[col / MH] = a0 + a1;
+  }
+}
+
 // Barrier over the epilogue warps (bounded; warp-uniform result).
 __device__ __forceinline__ bool ep_barrier(Smem& s, uint32_t& phase, uint32_t* status) {
   __syncwarp();
@@ -531,41 +553,33 @@ __global__ void __maxnreg__(96)
         const int buf = tb & 1;
         if (!(ok = warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status))) break;
         tc_fence_after();
+        // The warp's 64 columns in four 16-column TMEM loads, each issued
+        // before the previous chunk is summed, so the load latency overlaps
+        // the arithmetic; the buffer is released after the last load.
         const uint32_t taddr = lane_addr + buf * kN + half * kColsPerWarp;
+        const float* wcol = s.w + half * kColsPerWarp;
         float sc_[QH];
-        if constexpr (MH <= 32) {
-          // One 32-column load at a time: 32/MH whole queries per load.
-          constexpr int QPL = 32 / MH;
-#pragma unroll
-          for (int hh = 0; hh < kColsPerWarp / 32; ++hh) {
-            float v[32];
-            tmem_ld32(taddr + hh * 32, v);
-            tmem_wait_ld();
-            reg_fence32(v);
-            if (hh == kColsPerWarp / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&s.tempty[buf]);
-            }
-#pragma unroll
-            for (int q2 = 0; q2 < QPL; ++q2)
-              sc_[hh * QPL + q2] = relu_wsum<MH>([&](int j) { return v[q2 * MH + j]; },
-                                                 s.w + half * kColsPerWarp + hh * 32 + q2 * MH);
-          }
-        } else {
-          // MH == 64: the warp's one query spans both 32-column loads.
-          static_assert(MH != 64 || (QH == 1 && kColsPerWarp == 64), "one query per warp");
-          float v[2][32];
-          tmem_ld32(taddr, v[0]);
-          tmem_ld32(taddr + 32, v[1]);
-          tmem_wait_ld();
-          reg_fence32(v[0]);
-          reg_fence32(v[1]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[buf]);
-          sc_[0] = relu_wsum<MH>([&](int j) { return v[j >> 5][j & 31]; }, s.w + half * kColsPerWarp);
-        }
+        float a0 = 0.f, a1 = 0.f;
+        float vA[16], vB[16];
+        tmem_ld16(taddr, vA);
+        tmem_wait_ld();
+        reg_fence16(vA);
+        tmem_ld16(taddr + 16, vB);
+        chunk_wsum<MH, 0>(vA, wcol, a0, a1, sc_);
+        tmem_wait_ld();
+        reg_fence16(vB);
+        tmem_ld16(taddr + 32, vA);
+        chunk_wsum<MH, 1>(vB, wcol, a0, a1, sc_);
+        tmem_wait_ld();
+        reg_fence16(vA);
+        tmem_ld16(taddr + 48, vB);
+        chunk_wsum<MH, 2>(vA, wcol, a0, a1, sc_);
+        tmem_wait_ld();
+        reg_fence16(vB);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.tempty[buf]);
+        chunk_wsum<MH, 3>(vB, wcol, a0, a1, sc_);
         const int key = tile * kTileKeys + lrow;
         if (step == 0) {
           // Anchor every query's histogram at the maximum of its first tile.
