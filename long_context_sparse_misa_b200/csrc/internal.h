@@ -121,8 +121,8 @@ struct StreamArgs {
   int max_groups;
   int grid;               // persistent CTAs (<= number of SMs)
   int k;
-  uint2* cand;            // [grid * 32 queries * 4 quarters, subcap] candidate buffers
-  int64_t subcap;         // stream_subcap(max_seq_len)
+  uint2* cand;            // stream_cand_bytes(grid, subcap): candidate lists and counts
+  int64_t subcap;         // stream_subcap(max_seq_len): rows of each list
   int32_t* idx;
   float* val;
   int32_t* fail_list;     // [T] queries whose sampled threshold did not verify

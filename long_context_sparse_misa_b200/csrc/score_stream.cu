@@ -30,11 +30,11 @@
 //     of the prefix), i.e. a few standard deviations below the expected k-th
 //     best score.
 //   * main pass over all tiles: a key is appended to query q's candidates
-//     only if I >= tau_q.  Each (query, lane quarter) has a private
-//     sub-buffer with one slot per key the quarter can see, so nothing can
-//     overflow; per query, a ballot ranks the passing lanes and one
-//     predicated store writes them contiguously after the query's earlier
-//     appends (the running count is kept, warp-uniform, in registers).
+//     only if I >= tau_q.  Each (query, TMEM lane) has its own list with one
+//     row per tile, so nothing can overflow and no lane needs a rank from
+//     the others: a passing lane stores to row cnt of its list and counts
+//     (a predicated store and an add, no vote).  A query's 128 lists are
+//     stored row by row, so that a row of all lists is 1 KB contiguous.
 //   * check and select: every key scoring at least tau_q was appended, so if
 //     at least min(k, n) keys were appended the exact top-k is among them.
 //     The owner warp then histograms the candidates, takes those above the
@@ -72,7 +72,7 @@ constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 key
 // histograms (free by then).
 static_assert(kEpiWarps * kSelBins <= kMaxG * kBins, "select scratch must fit the histograms");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
-                           kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ + kMaxG * 4 * 4 /*wc*/ +
+                           kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ +
                            kMaxG * kBins * 4 /*hist, select*/ + 32 * 8 /*barriers*/ + 16;
 
 struct Smem {
@@ -84,7 +84,6 @@ struct Smem {
   float* tau;
   uint32_t* maxkey;
   int* base;  // histogram anchor per query
-  int* wc;    // [kMaxG][4] sub-buffer counts
   uint32_t* hist;
   uint32_t* sel;  // aliases hist
   uint64_t* full;
@@ -111,8 +110,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tau = reinterpret_cast<float*>(s.row + kMaxG);
   s.maxkey = reinterpret_cast<uint32_t*>(s.tau + kMaxG);
   s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
-  s.wc = s.base + kMaxG;
-  s.hist = reinterpret_cast<uint32_t*>(s.wc + kMaxG * 4);
+  s.hist = reinterpret_cast<uint32_t*>(s.base + kMaxG);
   s.sel = s.hist;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.hist + kMaxG * kBins);
   s.full = bars;
@@ -218,90 +216,105 @@ __device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint
   cnt_out = __shfl_sync(0xffffffffu, mc, src);
 }
 
-// Exact top-k of one query's four candidate sub-buffers (region[r*subcap ..],
-// counts cnt[r*cstride]), by one warp.  Threshold-bin entries are compacted
-// in order to the front of the region, which never overtakes the entries
-// still to be read.
-__device__ void final_select(uint2* region, int64_t subcap, const int* cnt, int cstride,
-                             const uint32_t* hist, int base, int k, int32_t* idx, float* val,
-                             uint32_t* selh) {
+// Exact top-k of one query's candidates, by one warp.  The candidates sit in
+// 128 lists (one per TMEM lane, i.e. per key row of a tile) stored row by
+// row: entry r of list l at region[r * 128 + l]; list l holds cnt[l]
+// entries.  Lane j reads lists j, j+32, j+64, j+96, so each load instruction
+// reads 256 contiguous bytes.  Threshold-bin entries are compacted to the
+// front of their own list, which only rewrites entries that the same lane
+// has already read.
+__device__ void final_select(uint2* region, const int* cnt, int base, int k, int32_t* idx,
+                             float* val, uint32_t* selh) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
-  int nr[4];
+  constexpr uint32_t kAll = 0xffffffffu;
+  int c[4], z[4];
+  int mine = 0, cm = 0;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) nr[r] = cnt[r * cstride];
-  const int n = nr[0] + nr[1] + nr[2] + nr[3];
+  for (int i = 0; i < 4; ++i) {
+    c[i] = cnt[lane + 32 * i];
+    z[i] = 0;
+    mine += c[i];
+    cm = max(cm, c[i]);
+  }
+  const int n = __reduce_add_sync(kAll, mine);
+  const int rows = __reduce_max_sync(kAll, cm);
+  uint2* mine_col = region + lane;  // entry (r, list lane + 32 i) at mine_col[r * 128 + 32 * i]
   int out = 0;
   if (n <= k) {
-    for (int r = 0; r < 4; ++r) {
-      const uint2* sb = region + r * subcap;
-      for (int j = lane; j < nr[r]; j += 32) {
-        const uint2 e = sb[j];
-        idx[out + j] = static_cast<int32_t>(e.y);
-        val[out + j] = __uint_as_float(e.x) + 0.0f;
+    for (int r = 0; r < rows; ++r) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool p = r < c[i];
+        uint2 e = make_uint2(0u, 0u);
+        if (p) e = mine_col[(int64_t)r * 128 + 32 * i];
+        const uint32_t b = __ballot_sync(kAll, p);
+        const int o = out + __popc(b & lt);
+        if (p) {
+          idx[o] = static_cast<int32_t>(e.y);
+          val[o] = __uint_as_float(e.x) + 0.0f;
+        }
+        out += __popc(b);
       }
-      out += nr[r];
     }
   } else {
+    constexpr int kR = 4;  // rows per batch: 16 loads in flight per lane
     // Pass 0: histogram of the entries (bins relative to the query's anchor).
-    constexpr int kH = 16;
     for (int i = lane; i < kBins; i += 32) selh[i] = 0u;
     __syncwarp();
-    for (int r = 0; r < 4; ++r) {
-      const uint2* sb = region + r * subcap;
-      for (int j0 = 0; j0 < nr[r]; j0 += 32 * kH) {
-        uint32_t xv[kH];
+    for (int r0 = 0; r0 < rows; r0 += kR) {
+      uint32_t xv[kR][4];
 #pragma unroll
-        for (int u = 0; u < kH; ++u) {
-          const int j = j0 + u * 32 + lane;
-          xv[u] = j < nr[r] ? __ldcs(&sb[j].x) : 0u;
-        }
+      for (int u = 0; u < kR; ++u)
 #pragma unroll
-        for (int u = 0; u < kH; ++u)
-          red_add_shared_if(&selh[score_bin(order_key(__uint_as_float(xv[u])), base)],
-                            j0 + u * 32 + lane < nr[r]);
-      }
+        for (int i = 0; i < 4; ++i)
+          xv[u][i] = r0 + u < c[i] ? __ldcs(&mine_col[(int64_t)(r0 + u) * 128 + 32 * i].x) : 0u;
+#pragma unroll
+      for (int u = 0; u < kR; ++u)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          red_add_shared_if(&selh[score_bin(order_key(__uint_as_float(xv[u][i])), base)],
+                            r0 + u < c[i]);
     }
     __syncwarp();
     int bstar;
     uint32_t A, Z;
-    find_crossing<4>(hist, kBins, (uint32_t)k, bstar, A, Z);
+    find_crossing<4>(selh, kBins, (uint32_t)k, bstar, A, Z);
     uint32_t need = (uint32_t)k - A;
     __syncwarp();
     // Pass 1: entries above the threshold bin go out; threshold-bin entries
-    // are compacted to the front of the region.  Each lane issues kU loads
-    // before using any of them (the buffer is mostly beyond L2).
-    constexpr int kU = 16;
-    int zpos = 0;
-    for (int r = 0; r < 4; ++r) {
-      const uint2* sb = region + r * subcap;
-      const int nrr = nr[r];
-      for (int j0 = 0; j0 < nrr; j0 += 32 * kU) {
-        uint2 ev[kU];
+    // move to the front of their list.
+    for (int r0 = 0; r0 < rows; r0 += kR) {
+      uint2 ev[kR][4];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int j = j0 + u * 32 + lane;
-          ev[u] = j < nrr ? __ldcs(sb + j) : make_uint2(0u, 0u);
-        }
-        __syncwarp();
+      for (int u = 0; u < kR; ++u)
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int j = j0 + u * 32 + lane;
-          const uint2 e = ev[u];
-          const int b = j < nrr ? score_bin(order_key(__uint_as_float(e.x)), base) : -1;
-          const uint32_t up = __ballot_sync(0xffffffffu, b > bstar);
+        for (int i = 0; i < 4; ++i)
+          ev[u][i] = r0 + u < c[i] ? __ldcs(&mine_col[(int64_t)(r0 + u) * 128 + 32 * i])
+                                   : make_uint2(0u, 0u);
+#pragma unroll
+      for (int u = 0; u < kR; ++u) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint2 e = ev[u][i];
+          const int b = r0 + u < c[i] ? score_bin(order_key(__uint_as_float(e.x)), base) : -1;
+          const uint32_t up = __ballot_sync(kAll, b > bstar);
           const int o = out + __popc(up & lt);
           st_global_u32_if(idx + o, e.y, b > bstar && o < k);
           st_global_u32_if(val + o, __float_as_uint(__uint_as_float(e.x) + 0.0f),
                            b > bstar && o < k);
           out += __popc(up);
-          const uint32_t zb = __ballot_sync(0xffffffffu, b == bstar);
-          st_global_u2_if(region + zpos + __popc(zb & lt), e.x, e.y, b == bstar);
-          zpos += __popc(zb);
+          if (b == bstar) {
+            mine_col[(int64_t)z[i] * 128 + 32 * i] = e;
+            ++z[i];
+          }
         }
-        __syncwarp();
       }
     }
+    int zm = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) zm = max(zm, z[i]);
+    const int zrows = __reduce_max_sync(kAll, zm);
     __syncwarp();
     // Pass 2: choose `need` of the Z threshold-bin entries by exact key.
     int shift = 64;
@@ -311,38 +324,41 @@ __device__ void final_select(uint2* region, int64_t subcap, const int* cnt, int 
         const int sh = 56 - 8 * p;
         for (int i = lane; i < kSelBins; i += 32) selh[i] = 0;
         __syncwarp();
-        for (int j = lane; j < (int)Z; j += 32) {
-          const uint64_t key = sel_key(region[j]);
-          if (p == 0 || (key >> (sh + 8)) == prefix) atomicAdd(&selh[(key >> sh) & 255u], 1u);
+        for (int r = 0; r < zrows; ++r) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (r < z[i]) {
+              const uint64_t key = sel_key(mine_col[(int64_t)r * 128 + 32 * i]);
+              if (p == 0 || (key >> (sh + 8)) == prefix) atomicAdd(&selh[(key >> sh) & 255u], 1u);
+            }
+          }
         }
         __syncwarp();
         int bin;
-        uint32_t ab, cnt;
-        find_crossing<8>(selh, kSelBins, need, bin, ab, cnt);
+        uint32_t ab, cn;
+        find_crossing<8>(selh, kSelBins, need, bin, ab, cn);
         need -= ab;
         prefix = (prefix << 8) | static_cast<uint64_t>(bin);
         shift = sh;
         __syncwarp();
-        if (cnt == need) break;
+        if (cn == need) break;
       }
     }
-    for (int j0 = 0; j0 < (int)Z; j0 += 32) {
-      const int j = j0 + lane;
-      bool take = false;
-      uint2 e = make_uint2(0u, 0u);
-      if (j < (int)Z) {
-        e = region[j];
-        take = shift == 64 || (sel_key(e) >> shift) >= prefix;
-      }
-      const uint32_t tb = __ballot_sync(0xffffffffu, take);
-      if (take) {
+    for (int r = 0; r < zrows; ++r) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool p = r < z[i];
+        uint2 e = make_uint2(0u, 0u);
+        if (p) e = mine_col[(int64_t)r * 128 + 32 * i];
+        const bool take = p && (shift == 64 || (sel_key(e) >> shift) >= prefix);
+        const uint32_t tb = __ballot_sync(kAll, take);
         const int o = out + __popc(tb & lt);
-        if (o < k) {
+        if (take && o < k) {
           idx[o] = static_cast<int32_t>(e.y);
           val[o] = __uint_as_float(e.x) + 0.0f;
         }
+        out += __popc(tb);
       }
-      out += __popc(tb);
     }
   }
   for (int j = out + lane; j < k; j += 32) {
@@ -502,7 +518,8 @@ __global__ void __maxnreg__(96)
     const int half = e >> 2;                 // column part: queries half*QH .. half*QH+QH-1
     const int lrow = quarter * 32 + lane;    // key row of the tile
     const int et = threadIdx.x - 64;         // 0..kEpiThreads-1
-    const uint32_t lt = (1u << lane) - 1u;
+    // Append counts per (CTA, query slot, list), after the candidate lists.
+    int* lcnt = reinterpret_cast<int*>(cand + (int64_t)gridDim.x * kMaxG * 128 * subcap);
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t ephase = 0;
     int tb = 0;
@@ -531,15 +548,13 @@ __global__ void __maxnreg__(96)
         s.maxkey[et] = 0u;
       }
       for (int i = et; i < G * kBins; i += kEpiThreads) s.hist[i] = 0u;
-      // This warp's slot counters (one per query; only this warp touches
-      // them) and its sub-buffer of its first query; query stride 4 * subcap.
-      int* mycnt = s.wc + quarter * kMaxG + half * QH;  // [quarter][query]
-      int cnt[QH];  // appends so far per query (warp-uniform)
+      // This lane's list of its warp's first query (row-major over the 128
+      // lists of a query) and its append counts, one per query.
+      uint2* mylist = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 128 * subcap + lrow;
+      const uint32_t qstride = 128u * static_cast<uint32_t>(subcap);
+      int cnt[QH];
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
-      uint2* mysub = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 4 * subcap +
-                     (int64_t)quarter * subcap;
-      const int qstride = 4 * static_cast<int>(subcap);
       if (!(ok = ep_barrier(s, ephase, status))) break;
       int minpos = 0x7fffffff;  // smallest valid position of the group (-1 if any invalid)
       for (int qi = 0; qi < nq; ++qi) minpos = min(minpos, s.pos[qi]);
@@ -642,25 +657,22 @@ __global__ void __maxnreg__(96)
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
         }
-        // Streaming selection: per query one ballot gives each passing lane
-        // its slot after the query's earlier appends (the count is the same
-        // in every lane of the warp), then one predicated 8-byte store per
-        // query writes the warp's appends contiguously.
+        // Streaming selection: a passing lane appends to its own list.
         // Tiles wholly below every query's position need no causal compare.
         const bool full_tile = (tile + 1) * kTileKeys <= minpos + 1;
 #pragma unroll
         for (int qq = 0; qq < QH; ++qq) {
           const bool take = (full_tile || key <= s.pos[half * QH + qq]) && sc_[qq] >= tauR[qq];
-          const uint32_t bq = __ballot_sync(0xffffffffu, take);
-          st_global_u2_if(mysub + (int64_t)qq * qstride + cnt[qq] + __popc(bq & lt),
+          st_global_u2_if(mylist + (qq * qstride + static_cast<uint32_t>(cnt[qq]) * 128u),
                           __float_as_uint(sc_[qq]), static_cast<uint32_t>(key), take);
-          cnt[qq] += __popc(bq);
+          cnt[qq] += take ? 1 : 0;
         }
       }
       if (!ok) break;
-      if (lane == 0) {
+      {
+        int* lc = lcnt + ((int64_t)blockIdx.x * kMaxG + half * QH) * 128 + lrow;
 #pragma unroll
-        for (int qq = 0; qq < QH; ++qq) mycnt[qq] = cnt[qq];
+        for (int qq = 0; qq < QH; ++qq) lc[qq * 128] = cnt[qq];
       }
       if (!(ok = ep_barrier(s, ephase, status))) break;
       for (int qi = e; qi < nq; qi += kEpiWarps) {
@@ -675,16 +687,16 @@ __global__ void __maxnreg__(96)
         // Verify the probe threshold: every key scoring at least the first
         // threshold was appended, so min(k, n) appended entries prove that the
         // exact top-k is among them.  Otherwise hand the query to the fixup.
-        const int napp = s.wc[qi] + s.wc[kMaxG + qi] + s.wc[2 * kMaxG + qi] +
-                         s.wc[3 * kMaxG + qi];
+        const int* qcnt = lcnt + ((int64_t)blockIdx.x * kMaxG + qi) * 128;
+        const int napp = __reduce_add_sync(0xffffffffu, qcnt[lane] + qcnt[lane + 32] +
+                                                            qcnt[lane + 64] + qcnt[lane + 96]);
         const int need = min(k, s.pos[qi] + 1);
         if (napp < need) {
           if (lane == 0 && sc.fail_out) sc.fail_out[atomicAdd(sc.fail_count, 1)] = t;
           continue;
         }
-        uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 4 * subcap;
-        final_select(region, subcap, s.wc + qi, kMaxG, s.sel + e * kSelBins,
-                     s.base[qi], k, idx_out + (int64_t)t * k,
+        uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 128 * subcap;
+        final_select(region, qcnt, s.base[qi], k, idx_out + (int64_t)t * k,
                      val_out + (int64_t)t * k, s.sel + e * kSelBins);
       }
       if (!(ok = ep_barrier(s, ephase, status))) break;
@@ -741,12 +753,13 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
 int stream_group_size(int m) { return kN / m; }
 
 int64_t stream_subcap(int max_seq_len) {
-  // keys one lane quarter can see: 32 per 128-key tile
-  return ((int64_t)max_seq_len + kTileKeys - 1) / kTileKeys * 32;
+  // rows of a lane's list: one per 128-key tile of the longest prefix
+  return ((int64_t)max_seq_len + kTileKeys - 1) / kTileKeys;
 }
 
 size_t stream_cand_bytes(int grid, int64_t subcap) {
-  return (size_t)grid * kMaxG * 4 * (size_t)subcap * sizeof(uint2);
+  // lists [grid][kMaxG][subcap rows][128], then counts [grid][kMaxG][128]
+  return (size_t)grid * kMaxG * 128 * ((size_t)subcap * sizeof(uint2) + sizeof(int));
 }
 
 int launch_score_stream(const StreamArgs& a, cudaStream_t st) {
