@@ -23,8 +23,10 @@
 // I = sum_j w_j ReLU(acc_j) (the TMEM buffer is released after the warp's
 // last load), the causal mask, and the streaming selection:
 //   * probe: a group first scores every 8th tile of its prefix and keeps a
-//     128-bin histogram per query (1/8-octave bins of the order-preserving
-//     score key, anchored 14 octaves below the first scored tile's maximum).
+//     128-bin histogram per query (1/16-octave bins of the order-preserving
+//     score key, from 6 octaves below the first scored tile's maximum to 2
+//     above; scores outside fall into the end bins, which can only lower the
+//     threshold).
 //     The starting threshold tau_q is the lower edge of the bin holding the
 //     r-th best sampled score, r = k*f + 4*sqrt(k*f) + 1 (f = sampled share
 //     of the prefix), i.e. a few standard deviations below the expected k-th
@@ -61,8 +63,8 @@ constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kTmemCols = 2 * kN;
 constexpr int kMaxG = 32;                        // queries per group (m >= 8)
 constexpr int kBins = 128;
-constexpr int kBinShift = 20;                    // 12-bit score key prefix: 1/8 octave
-constexpr int kHeadroom = 112;                   // bins below the first tile's maximum
+constexpr int kBinShift = 19;                    // 13-bit score key prefix: 1/16 octave
+constexpr int kHeadroom = 96;                    // bins below the first tile's maximum
 constexpr int kSelBins = 256;
 constexpr int kProbeStride = 8;                  // probe every 8th tile ...
 constexpr int kProbeOff = 4;                     // ... starting at tile 4
@@ -126,7 +128,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-// Histogram anchor of a query: 14 octaves below its first tile's maximum.
+// Histogram anchor of a query: 6 octaves below its first tile's maximum.
 __device__ __forceinline__ int hist_base(uint32_t maxkey) {
   const int b = static_cast<int>(maxkey >> kBinShift) - kHeadroom;
   return b < 0 ? 0 : b;
