@@ -272,6 +272,13 @@ __device__ __forceinline__ void red_add_shared_if(uint32_t* p, bool pred) {
       "r"((int)pred)
       : "memory");
 }
+__device__ __forceinline__ void red_add_shared_val_if(uint32_t* p, uint32_t v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q red.shared.add.u32 [%0], %1;\n\t}\n" ::"r"(
+          smem_u32(p)),
+      "r"(v), "r"((int)pred)
+      : "memory");
+}
 __device__ __forceinline__ void st_global_u2_if(void* p, uint32_t x, uint32_t y, bool pred) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t@q st.global.v2.u32 [%0], {%1, %2};\n\t}\n" ::"l"(

@@ -23,10 +23,10 @@
 // I = sum_j w_j ReLU(acc_j) (the TMEM buffer is released after the warp's
 // last load), the causal mask, and the streaming selection:
 //   * probe: a group first scores every 8th tile of its prefix and keeps a
-//     128-bin histogram per query (1/16-octave bins of the order-preserving
-//     score key, from 6 octaves below the first scored tile's maximum to 2
+//     256-bin histogram per query (1/32-octave bins of the order-preserving
+//     score key, from 7 octaves below the first scored tile's maximum to one
 //     above; scores outside fall into the end bins, which can only lower the
-//     threshold).
+//     threshold).  Two 16-bit counts per shared word.
 //     The starting threshold tau_q is the lower edge of the bin holding the
 //     r-th best sampled score, r = k*f + 4*sqrt(k*f) + 1 (f = sampled share
 //     of the prefix), i.e. a few standard deviations below the expected k-th
@@ -62,9 +62,10 @@ constexpr int kQHalfBytes = kN * 128;            // 32 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kTmemCols = 2 * kN;
 constexpr int kMaxG = 32;                        // queries per group (m >= 8)
-constexpr int kBins = 128;
-constexpr int kBinShift = 19;                    // 13-bit score key prefix: 1/16 octave
-constexpr int kHeadroom = 96;                    // bins below the first tile's maximum
+constexpr int kBins = 256;
+constexpr int kHistWords = kBins / 2;            // two 16-bit bin counts per word
+constexpr int kBinShift = 18;                    // 14-bit score key prefix: 1/32 octave
+constexpr int kHeadroom = 224;                   // bins below the first tile's maximum
 constexpr int kSelBins = 256;
 constexpr int kProbeStride = 8;                  // probe every 8th tile ...
 constexpr int kProbeOff = 4;                     // ... starting at tile 4
@@ -72,10 +73,11 @@ constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 key
 
 // The per-warp select scratch of the final selection reuses the probe
 // histograms (free by then).
-static_assert(kEpiWarps * kSelBins <= kMaxG * kBins, "select scratch must fit the histograms");
+static_assert(kEpiWarps * kSelBins <= kMaxG * kHistWords, "select scratch must fit the histograms");
+static_assert(kSelBins >= kBins, "final-select histogram");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
                            kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ +
-                           kMaxG * kBins * 4 /*hist, select*/ + 32 * 8 /*barriers*/ + 16;
+                           kMaxG * kHistWords * 4 /*hist, select*/ + 32 * 8 /*barriers*/ + 16;
 
 struct Smem {
   uint8_t* q;
@@ -114,7 +116,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
   s.hist = reinterpret_cast<uint32_t*>(s.base + kMaxG);
   s.sel = s.hist;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.hist + kMaxG * kBins);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.hist + kMaxG * kHistWords);
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
@@ -128,7 +130,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-// Histogram anchor of a query: 6 octaves below its first tile's maximum.
+// Histogram anchor of a query: 7 octaves below its first tile's maximum.
 __device__ __forceinline__ int hist_base(uint32_t maxkey) {
   const int b = static_cast<int>(maxkey >> kBinShift) - kHeadroom;
   return b < 0 ? 0 : b;
@@ -178,14 +180,14 @@ __device__ __forceinline__ uint64_t sel_key(uint2 e) {
 
 // Bin (of `nb` descending-ordered counts, `per` per lane) where the count
 // from the top reaches `need`; returns bin, count above it and its count.
-template <int PER>
-__device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint32_t need,
-                                              int& bin, uint32_t& above_out, uint32_t& cnt_out) {
+template <int PER, typename Count>
+__device__ __forceinline__ void find_crossing_by(Count count, int nb, uint32_t need, int& bin,
+                                                 uint32_t& above_out, uint32_t& cnt_out) {
   const int lane = threadIdx.x & 31;
   uint32_t c[PER], loc = 0;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
-    c[i] = hist[nb - 1 - (lane * PER + i)];
+    c[i] = count(nb - 1 - (lane * PER + i));
     loc += c[i];
   }
   uint32_t inc = loc;
@@ -216,6 +218,21 @@ __device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint
   bin = __shfl_sync(0xffffffffu, mb, src);
   above_out = __shfl_sync(0xffffffffu, ma, src);
   cnt_out = __shfl_sync(0xffffffffu, mc, src);
+}
+
+template <int PER>
+__device__ __forceinline__ void find_crossing(const uint32_t* hist, int nb, uint32_t need,
+                                              int& bin, uint32_t& above_out, uint32_t& cnt_out) {
+  find_crossing_by<PER>([&](int b) { return hist[b]; }, nb, need, bin, above_out, cnt_out);
+}
+
+// Same over a histogram of 16-bit counts packed two per word.
+template <int PER>
+__device__ __forceinline__ void find_crossing16(const uint32_t* words, int nb, uint32_t need,
+                                                int& bin, uint32_t& above_out,
+                                                uint32_t& cnt_out) {
+  find_crossing_by<PER>([&](int b) { return (words[b >> 1] >> ((b & 1) * 16)) & 0xffffu; }, nb,
+                        need, bin, above_out, cnt_out);
 }
 
 // Exact top-k of one query's candidates, by one warp.  The candidates sit in
@@ -281,7 +298,7 @@ __device__ void final_select(uint2* region, const int* cnt, int base, int k, int
     __syncwarp();
     int bstar;
     uint32_t A, Z;
-    find_crossing<4>(selh, kBins, (uint32_t)k, bstar, A, Z);
+    find_crossing<kBins / 32>(selh, kBins, (uint32_t)k, bstar, A, Z);
     uint32_t need = (uint32_t)k - A;
     __syncwarp();
     // Pass 1: entries above the threshold bin go out; threshold-bin entries
@@ -390,9 +407,12 @@ __device__ __forceinline__ int4 fetch_group(const Sched& sc, int count, int gs) 
 
 // Probe schedule: tiles kProbeOff, kProbeOff + kProbeStride, ... of groups
 // whose longest prefix spans at least kProbeMinTiles tiles.
+// At most kProbeMaxTiles, so that no 16-bit bin count can overflow.
+constexpr int kProbeMaxTiles = 65535 / kTileKeys;
 __device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
-  return (probe && ntiles >= kProbeMinTiles) ? (ntiles - kProbeOff + kProbeStride - 1) / kProbeStride
-                                             : 0;
+  if (!probe || ntiles < kProbeMinTiles) return 0;
+  const int np = (ntiles - kProbeOff + kProbeStride - 1) / kProbeStride;
+  return np < kProbeMaxTiles ? np : kProbeMaxTiles;
 }
 
 template <int MH>
@@ -549,7 +569,7 @@ __global__ void __maxnreg__(96)
         s.tau[et] = p >= 0 ? -INFINITY : INFINITY;  // padding / invalid slots never append
         s.maxkey[et] = 0u;
       }
-      for (int i = et; i < G * kBins; i += kEpiThreads) s.hist[i] = 0u;
+      for (int i = et; i < G * kHistWords; i += kEpiThreads) s.hist[i] = 0u;
       // This lane's list of its warp's first query (row-major over the 128
       // lists of a query) and its append counts, one per query.
       uint2* mylist = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 128 * subcap + lrow;
@@ -617,8 +637,9 @@ __global__ void __maxnreg__(96)
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) {
             const int qi = half * QH + qq;
-            red_add_shared_if(&s.hist[qi * kBins + score_bin(order_key(sc_[qq]), s.base[qi])],
-                              key <= s.pos[qi]);
+            const int b = score_bin(order_key(sc_[qq]), s.base[qi]);
+            red_add_shared_val_if(&s.hist[qi * kHistWords + (b >> 1)], 1u << ((b & 1) * 16),
+                                  key <= s.pos[qi]);
           }
           if (step == np - 1) {
             // Starting thresholds from the sample: the bin holding the r-th
@@ -640,13 +661,14 @@ __global__ void __maxnreg__(96)
                 if (r <= ns) {
                   int bstar;
                   uint32_t A, Z;
-                  find_crossing<4>(s.hist + qi * kBins, kBins, (uint32_t)r, bstar, A, Z);
+                  find_crossing16<kBins / 32>(s.hist + qi * kHistWords, kBins, (uint32_t)r, bstar,
+                                              A, Z);
                   if (bstar > 0)
                     t0 = key_to_float(static_cast<uint32_t>(s.base[qi] + bstar) << kBinShift);
                 }
               }
               if (lane == 0) s.tau[qi] = t0;
-              for (int b = lane; b < kBins; b += 32) s.hist[qi * kBins + b] = 0u;
+              for (int b = lane; b < kHistWords; b += 32) s.hist[qi * kHistWords + b] = 0u;
             }
             if (!(ok = ep_barrier(s, ephase, status))) break;
 #pragma unroll
