@@ -236,14 +236,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int qi = 1; qi < nq; ++qi) consec &= (s.pos[qi] == s.pos[0] + qi) && s.pos[qi] >= 0;
       consec &= s.pos[0] >= 0;
       if (consec) {
+        // Running block sums in key order; 16 loads in flight per thread.
         const int p0 = s.pos[0], p1 = s.pos[nq - 1];
+        const int k0 = (p0 / B) * B;
         float run = 0.f;
-        for (int key = (p0 / B) * B; key <= p1; ++key) {
-          if (key % B == 0) run = 0.f;
-          run += bf16_bits_to_float(Kseq[(int64_t)key * kD]);
-          if (key >= p0) {
-            const int cntv = key - (key / B) * B + 1;
-            s.P[(key - p0) * kD + d] = run / (float)cntv;
+        for (int kb = k0; kb <= p1; kb += 16) {
+          float x[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            x[u] = kb + u <= p1 ? bf16_bits_to_float(Kseq[(int64_t)(kb + u) * kD]) : 0.f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int key = kb + u;
+            if (key > p1) break;
+            if (key % B == 0) run = 0.f;
+            run += x[u];
+            if (key >= p0) {
+              const int cntv = key - (key / B) * B + 1;
+              s.P[(key - p0) * kD + d] = run / (float)cntv;
+            }
           }
         }
       } else {
