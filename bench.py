@@ -148,17 +148,24 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  The
+    data path has no collective: each rank runs its own problem; the process
+    group only carries the barriers and the max-over-ranks of the timings.
+    backend "gloo" (CPU) is used by the multi-rank tests."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl" and torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -170,13 +177,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(cfg: int, rank: int) -> int:
+    """Seed of rank `rank`'s problem: every rank scores its own independent
+    problem of the same shape (weak scaling)."""
+    return 1000 + cfg + 100 * rank
+
+
+def job_throughput(units_per_rank: int, world: int, ms_step_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_step_max / 1e3)
 
 
 def workload_config(wl, cfg):
@@ -268,7 +288,7 @@ def run_ours(args):
 
     world, rank, local = dist_init()
     cfg = args.config
-    wl = make_config(cfg, seed=1000 + cfg + 100 * rank)
+    wl = make_config(cfg, seed=rank_seed(cfg, rank))
     if args.max_queries and args.max_queries < wl.T:
         wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
     hier = bool(wl.k_cand)
@@ -321,7 +341,7 @@ def run_ours(args):
         raise RuntimeError(f"device status {code} ({bits}) in the timed region")
     ms_step = ms / args.steps
     pairs = wl.pairs
-    value = pairs * world / (ms_step / 1e3)
+    value = job_throughput(pairs, world, ms_step)
 
     # ---- roofline of the dominant kernel (routed scoring on tcgen05)
     peaks = load_peaks()
@@ -380,7 +400,7 @@ def run_ours(args):
         dms = max_over_ranks(sum(a.elapsed_time(b) for a, b in devs), world) / dense_steps
         d_k_ms = dprof.get("score", (float("nan"), 0))[0] / dense_steps
         d_flops = 2.0 * wl.H * wl.d * pairs
-        line["dense_dsa"] = {"ms_per_step": dms, "value": pairs * world / (dms / 1e3),
+        line["dense_dsa"] = {"ms_per_step": dms, "value": job_throughput(pairs, world, dms),
                              "unit": UNIT, "misa_speedup": dms / ms_step,
                              "score_kernel_tflops": d_flops / (d_k_ms / 1e3) / 1e12,
                              "score_kernel_frac": d_flops / (d_k_ms / 1e3) / 1e12 / peaks["bf16_sustained"]}
@@ -411,7 +431,7 @@ def run_ours(args):
         e1.record()
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-        line["e2e"] = {"value": pairs * world / (ems / 1e3), "unit": UNIT,
+        line["e2e"] = {"value": job_throughput(pairs, world, ems), "unit": UNIT,
                        "ms_per_step": ems,
                        "h2d_bytes_per_step": K_h.nbytes + q_h.nbytes + w_h.nbytes,
                        "d2h_bytes_per_step": idx_h.nbytes + val_h.nbytes}
