@@ -37,12 +37,17 @@
 //     the others: a passing lane stores to row cnt of its list and counts
 //     (a predicated store and an add, no vote).  A query's 128 lists are
 //     stored row by row, so that a row of all lists is 1 KB contiguous.
-//   * check and select: every key scoring at least tau_q was appended, so if
-//     at least min(k, n) keys were appended the exact top-k is among them.
-//     The owner warp then histograms the candidates, takes those above the
-//     bin holding the k-th, and resolves that bin with a warp-level radix
-//     select over (score, lower index first).  A query with too few
-//     candidates is listed and rescanned by a second launch without a probe.
+//   * check and select, by two selector warps while the epilogue warps
+//     already stream the next group (the candidate lists are double
+//     buffered; when the selectors fall behind, the epilogue warps claim the
+//     remaining queries of the older buffer before reusing it): every key
+//     scoring at least tau_q was appended, so if at
+//     least min(k, n) keys were appended (and no list ran past its rows) the
+//     exact top-k is among them.  The selector then histograms the
+//     candidates, takes those above the bin holding the k-th, and resolves
+//     that bin with a warp-level radix select over (score, lower index
+//     first).  A query that fails the check is listed and rescanned by a
+//     second launch without a probe, with lists of one row per tile.
 #include "common.cuh"
 #include "internal.h"
 
@@ -55,7 +60,13 @@ constexpr int kHalfBytes = kStageBytes / 2;
 constexpr int kN = 256;                          // MMA N = group columns
 constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kThreads = 64 + kEpiThreads;       // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
+// Final selection, one group behind.  Registers are split evenly over the
+// four SM sub-partitions (16K each) and warps go to them round-robin, so 20
+// warps (five per sub-partition) is the most that fits at 96 registers.
+constexpr int kSelWarps = 2;
+// warp 0 TMA, warp 1 MMA, warps 2..17 epilogue, warps 18..19 selectors
+constexpr int kThreads = 64 + kEpiThreads + 32 * kSelWarps;
+constexpr int kRowsCap = 128;                    // rows per candidate list (main pass)
 constexpr int kParts = kEpiWarps / 4;            // column parts per TMEM lane quarter
 constexpr int kColsPerWarp = kN / kParts;
 constexpr int kQHalfBytes = kN * 128;            // 32 KB per 64-dim half
@@ -71,13 +82,13 @@ constexpr int kProbeStride = 8;                  // probe every 8th tile ...
 constexpr int kProbeOff = 4;                     // ... starting at tile 4
 constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
 
-// The per-warp select scratch of the final selection reuses the probe
-// histograms (free by then).
-static_assert(kEpiWarps * kSelBins <= kMaxG * kHistWords, "select scratch must fit the histograms");
 static_assert(kSelBins >= kBins, "final-select histogram");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
                            kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ +
-                           kMaxG * kHistWords * 4 /*hist, select*/ + 32 * 8 /*barriers*/ + 16;
+                           kMaxG * kHistWords * 4 /*hist*/ + kSelWarps * kSelBins * 4 /*select*/ +
+                           2 * kMaxG * 4 * 3 /*selector copies of pos,row,base*/ +
+                           2 * 4 * 3 /*selnq,selnext,seldone*/ +
+                           32 * 8 /*barriers*/ + 16;
 
 struct Smem {
   uint8_t* q;
@@ -89,7 +100,14 @@ struct Smem {
   uint32_t* maxkey;
   int* base;  // histogram anchor per query
   uint32_t* hist;
-  uint32_t* sel;  // aliases hist
+  uint32_t* sel;   // [kSelWarps][kSelBins]
+  int* mpos;       // [2][kMaxG] the selectors' copies of pos, row, base
+  int* mrow;
+  int* mbase;
+  int* selnq;          // [2] queries of the group in each candidate buffer
+  int* selnext;        // [2] next query to claim for selection
+  int* seldone;        // [2] queries selected
+  uint64_t* selready;  // [2] a group's candidates are complete
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -115,8 +133,14 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.maxkey = reinterpret_cast<uint32_t*>(s.tau + kMaxG);
   s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
   s.hist = reinterpret_cast<uint32_t*>(s.base + kMaxG);
-  s.sel = s.hist;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.hist + kMaxG * kHistWords);
+  s.sel = s.hist + kMaxG * kHistWords;
+  s.mpos = reinterpret_cast<int*>(s.sel + kSelWarps * kSelBins);
+  s.mrow = s.mpos + 2 * kMaxG;
+  s.mbase = s.mrow + 2 * kMaxG;
+  s.selnq = s.mbase + 2 * kMaxG;
+  s.selnext = s.selnq + 2;
+  s.seldone = s.selnext + 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.seldone + 2);
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
@@ -125,7 +149,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.qempty = s.qfull + 1;
   s.ebar = s.qempty + 1;
   s.drain = s.ebar + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.selready = s.drain + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.selready + 2);
   s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
   return s;
 }
@@ -415,14 +440,100 @@ __device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
   return np < kProbeMaxTiles ? np : kProbeMaxTiles;
 }
 
+// Candidate list of (buffer b, query slot q) of this CTA: rows_cap rows of 128.
+struct Lists {
+  uint2* cand;   // [grid][2][slots][rows_cap][128]
+  int* cnt;      // [grid][2][slots][128]
+  int rows_cap;
+  int slots;
+  __device__ __forceinline__ int64_t id(int b, int q) const {
+    return ((int64_t)blockIdx.x * 2 + b) * slots + q;
+  }
+  __device__ __forceinline__ uint2* list(int b, int q) const {
+    return cand + id(b, q) * rows_cap * 128;
+  }
+  __device__ __forceinline__ int* counts(int b, int q) const { return cnt + id(b, q) * 128; }
+};
+
+// Verify one query of a handed-over group and select its exact top-k (one
+// warp).  Every key scoring at least the starting threshold was appended, so
+// min(k, n) appended entries (none dropped at a full list) prove that the
+// exact top-k is among them; otherwise the query goes to the rescan launch.
+__device__ void select_query(const Smem& s, const Lists& ls, const Sched& sc, int b, int qi,
+                             int k, int32_t* idx_out, float* val_out, uint32_t* selh) {
+  const int lane = threadIdx.x & 31;
+  const int t = s.mrow[b * kMaxG + qi];
+  const int p = s.mpos[b * kMaxG + qi];
+  if (p < 0) {  // invalid position: padded row
+    for (int j = lane; j < k; j += 32) {
+      idx_out[(int64_t)t * k + j] = -1;
+      val_out[(int64_t)t * k + j] = -INFINITY;
+    }
+    return;
+  }
+  const int* qcnt = ls.counts(b, qi);
+  const int c0 = qcnt[lane], c1 = qcnt[lane + 32], c2 = qcnt[lane + 64], c3 = qcnt[lane + 96];
+  const int napp = __reduce_add_sync(0xffffffffu, c0 + c1 + c2 + c3);
+  const int cmax = __reduce_max_sync(0xffffffffu, max(max(c0, c1), max(c2, c3)));
+  const int need = min(k, p + 1);
+  if (napp < need || cmax > ls.rows_cap) {
+    if (lane == 0 && sc.fail_out) sc.fail_out[atomicAdd(sc.fail_count, 1)] = t;
+    return;
+  }
+  final_select(ls.list(b, qi), qcnt, s.mbase[b * kMaxG + qi], k, idx_out + (int64_t)t * k,
+               val_out + (int64_t)t * k, selh);
+}
+
+// Claims queries of candidate buffer b and selects them until none is left.
+__device__ void select_claimed(const Smem& s, const Lists& ls, const Sched& sc, int b, int nq,
+                               int k, int32_t* idx_out, float* val_out, uint32_t* selh) {
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    int qi = 0;
+    if (lane == 0) qi = atomicAdd(&s.selnext[b], 1);
+    qi = __shfl_sync(0xffffffffu, qi, 0);
+    if (qi >= nq) break;
+    select_query(s, ls, sc, b, qi, k, idx_out, val_out, selh);
+    __syncwarp();
+    __threadfence_block();  // this warp's reads of the lists are done
+    if (lane == 0) atomicAdd(&s.seldone[b], 1);
+  }
+}
+
+// Bounded wait (warp-uniform) until *c >= target.
+__device__ __forceinline__ bool wait_count(const int* c, int target, int* abort,
+                                           uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const long long t0 = clock64();
+  while (true) {
+    int v = 0, give_up = 0;
+    if (lane == 0) {
+      v = *reinterpret_cast<const volatile int*>(c);
+      if (v < target) {
+        if (*reinterpret_cast<volatile int*>(abort)) {
+          give_up = 1;
+        } else if (clock64() - t0 > kWaitCycles) {
+          *reinterpret_cast<volatile int*>(abort) = 1;
+          set_status(status, MISA_STATUS_TIMEOUT);
+          give_up = 1;
+        }
+      }
+    }
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v >= target) return true;
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+    __nanosleep(128);
+  }
+}
+
 template <int MH>
-// 18 warps at 96 registers each: one CTA per SM.
+// 20 warps at 96 registers each: one CTA per SM.
 __global__ void __maxnreg__(96)
     score_stream_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap qmap, const float* __restrict__ wsel,
-                        const int64_t* __restrict__ ko, Sched sc, int k, uint2* __restrict__ cand,
-                        int64_t subcap, int32_t* __restrict__ idx_out,
-                        float* __restrict__ val_out, uint32_t* status) {
+                        const int64_t* __restrict__ ko, Sched sc, int k, Lists ls,
+                        int32_t* __restrict__ idx_out, float* __restrict__ val_out,
+                        uint32_t* status) {
   constexpr int G = kN / MH;          // queries per group
   constexpr int QH = G / kParts;      // queries per epilogue warp (its column part)
   static_assert(MH >= 8 && MH <= 64 && G <= kMaxG && QH >= 1, "unsupported head count");
@@ -448,6 +559,9 @@ __global__ void __maxnreg__(96)
     mbar_init(s.qempty, 1);
     mbar_init(s.ebar, kEpiWarps);
     mbar_init(s.drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.selready[i], kEpiWarps);
+    }
     *s.abort = 0;
     fence_barrier_init();
   }
@@ -533,15 +647,14 @@ __global__ void __maxnreg__(96)
       umma_commit(s.drain);
       mbar_wait(s.drain, 0, s.abort, status, kDrainCycles, true);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;                  // 0..kEpiWarps-1
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
     const int half = e >> 2;                 // column part: queries half*QH .. half*QH+QH-1
     const int lrow = quarter * 32 + lane;    // key row of the tile
     const int et = threadIdx.x - 64;         // 0..kEpiThreads-1
-    // Append counts per (CTA, query slot, list), after the candidate lists.
-    int* lcnt = reinterpret_cast<int*>(cand + (int64_t)gridDim.x * kMaxG * 128 * subcap);
+    int gl = 0;  // groups done by this warp (candidate buffer gl & 1)
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t ephase = 0;
     int tb = 0;
@@ -553,6 +666,16 @@ __global__ void __maxnreg__(96)
       const int ntiles = (grp.w + kTileKeys) / kTileKeys;
       const int np = probe_tiles(probe, ntiles);
       const int64_t L = ko[seq + 1] - ko[seq];
+      const int bsel = gl & 1;
+      if (gl >= 2) {
+        // The group two back used this candidate buffer: claim what the
+        // selectors have not taken yet, then wait until all of it is done.
+        // The probe histograms are free here and serve as select scratch.
+        const int nqo = s.selnq[bsel];
+        select_claimed(s, ls, sc, bsel, nqo, k, idx_out, val_out, s.hist + e * kSelBins);
+        if (!(ok = wait_count(&s.seldone[bsel], nqo, s.abort, status))) break;
+        if (!(ok = ep_barrier(s, ephase, status))) break;
+      }
       // Group state: column weights, query limits, selection state.
       if (et < kN) {
         const int qi = et / MH;
@@ -572,8 +695,9 @@ __global__ void __maxnreg__(96)
       for (int i = et; i < G * kHistWords; i += kEpiThreads) s.hist[i] = 0u;
       // This lane's list of its warp's first query (row-major over the 128
       // lists of a query) and its append counts, one per query.
-      uint2* mylist = cand + ((int64_t)blockIdx.x * kMaxG + half * QH) * 128 * subcap + lrow;
-      const uint32_t qstride = 128u * static_cast<uint32_t>(subcap);
+      uint2* mylist = ls.list(bsel, 0) + (int64_t)(half * QH) * ls.rows_cap * 128 + lrow;
+      const uint32_t qstride = 128u * static_cast<uint32_t>(ls.rows_cap);
+      const int rows_cap = ls.rows_cap;
       int cnt[QH];
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
@@ -688,42 +812,53 @@ __global__ void __maxnreg__(96)
         for (int qq = 0; qq < QH; ++qq) {
           const bool take = (full_tile || key <= s.pos[half * QH + qq]) && sc_[qq] >= tauR[qq];
           st_global_u2_if(mylist + (qq * qstride + static_cast<uint32_t>(cnt[qq]) * 128u),
-                          __float_as_uint(sc_[qq]), static_cast<uint32_t>(key), take);
-          cnt[qq] += take ? 1 : 0;
+                          __float_as_uint(sc_[qq]), static_cast<uint32_t>(key),
+                          take && cnt[qq] < rows_cap);
+          cnt[qq] += take ? 1 : 0;  // counts past rows_cap mark the list as overflowed
         }
       }
       if (!ok) break;
-      {
-        int* lc = lcnt + ((int64_t)blockIdx.x * kMaxG + half * QH) * 128 + lrow;
+      // Hand the group to the selectors: counts, and (warp 0 of the
+      // epilogue) the per-query positions, rows and histogram anchors.
 #pragma unroll
-        for (int qq = 0; qq < QH; ++qq) lc[qq * 128] = cnt[qq];
-      }
-      if (!(ok = ep_barrier(s, ephase, status))) break;
-      for (int qi = e; qi < nq; qi += kEpiWarps) {
-        const int t = s.row[qi];
-        if (s.pos[qi] < 0) {  // invalid position: padded row
-          for (int j = lane; j < k; j += 32) {
-            idx_out[(int64_t)t * k + j] = -1;
-            val_out[(int64_t)t * k + j] = -INFINITY;
-          }
-          continue;
+      for (int qq = 0; qq < QH; ++qq)
+        if (half * QH + qq < nq) ls.counts(bsel, half * QH + qq)[lrow] = cnt[qq];
+      if (e == 0) {
+        s.mpos[bsel * kMaxG + lane] = lane < G ? s.pos[lane] : -1;
+        s.mrow[bsel * kMaxG + lane] = lane < G ? s.row[lane] : 0;
+        s.mbase[bsel * kMaxG + lane] = lane < G ? s.base[lane] : 0;
+        if (lane == 0) {
+          s.selnq[bsel] = nq;
+          s.selnext[bsel] = 0;
+          s.seldone[bsel] = 0;
         }
-        // Verify the probe threshold: every key scoring at least the first
-        // threshold was appended, so min(k, n) appended entries prove that the
-        // exact top-k is among them.  Otherwise hand the query to the fixup.
-        const int* qcnt = lcnt + ((int64_t)blockIdx.x * kMaxG + qi) * 128;
-        const int napp = __reduce_add_sync(0xffffffffu, qcnt[lane] + qcnt[lane + 32] +
-                                                            qcnt[lane + 64] + qcnt[lane + 96]);
-        const int need = min(k, s.pos[qi] + 1);
-        if (napp < need) {
-          if (lane == 0 && sc.fail_out) sc.fail_out[atomicAdd(sc.fail_count, 1)] = t;
-          continue;
-        }
-        uint2* region = cand + ((int64_t)blockIdx.x * kMaxG + qi) * 128 * subcap;
-        final_select(region, qcnt, s.base[qi], k, idx_out + (int64_t)t * k,
-                     val_out + (int64_t)t * k, s.sel + e * kSelBins);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.selready[bsel]);
+      ++gl;
       if (!(ok = ep_barrier(s, ephase, status))) break;
+    }
+    // Help the selectors with the last groups (no more probing: the
+    // histograms are free).
+    for (int j = gl >= 2 ? gl - 2 : 0; ok && j < gl; ++j)
+      select_claimed(s, ls, sc, j & 1, s.selnq[j & 1], k, idx_out, val_out,
+                     s.hist + e * kSelBins);
+  } else {
+    // ------------------------------------------------------------ selectors
+    // Verify each query of the previous group and select its exact top-k
+    // from the candidates, while the epilogue streams the next group.
+    const int sw = warp - 2 - kEpiWarps;  // 0..kSelWarps-1
+    uint32_t* selh = s.sel + sw * kSelBins;
+    int gl = 0;
+    bool ok = true;
+    for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+      const int4 grp = fetch_group(sc, count, gs);
+      if (grp.w < 0) continue;
+      const int nq = grp.z - grp.y;
+      const int bsel = gl & 1;
+      if (!(ok = warp_wait(&s.selready[bsel], (gl >> 1) & 1, s.abort, status))) break;
+      select_claimed(s, ls, sc, bsel, nq, k, idx_out, val_out, selh);
+      ++gl;
     }
   }
 
@@ -736,15 +871,36 @@ __global__ void __maxnreg__(96)
   }
 }
 
+// Candidate storage (one workspace region, 256-byte aligned parts): the main
+// pass's lists [grid][2][kMaxG][rows_main][128] and counts, then the rescan's
+// lists [grid][2][1][rows_full][128] and counts.
+struct CandLayout {
+  int rows_main, rows_full;
+  size_t main_lists, main_counts, fix_lists, fix_counts;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+CandLayout cand_layout(int grid, int64_t rows_full) {
+  CandLayout c;
+  c.rows_full = (int)rows_full;
+  c.rows_main = rows_full < kRowsCap ? (int)rows_full : kRowsCap;
+  c.main_lists = align256((size_t)grid * 2 * kMaxG * c.rows_main * 128 * sizeof(uint2));
+  c.main_counts = align256((size_t)grid * 2 * kMaxG * 128 * sizeof(int));
+  c.fix_lists = align256((size_t)grid * 2 * c.rows_full * 128 * sizeof(uint2));
+  c.fix_counts = align256((size_t)grid * 2 * 128 * sizeof(int));
+  return c;
+}
+
 template <int MH>
 int launch_one(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap& qmap,
-               const Sched& sc, cudaStream_t st) {
+               const Sched& sc, const Lists& ls, cudaStream_t st) {
   auto kern = score_stream_kernel<MH>;
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
   ProfScope ps(sc.fail_in ? "score_fixup" : "score", st);
-  kern<<<a.grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.wsel, a.p->key_offsets, sc, a.k,
-                                            a.cand, a.subcap, a.idx, a.val, status_ptr());
+  kern<<<a.grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.wsel, a.p->key_offsets, sc, a.k, ls,
+                                            a.idx, a.val, status_ptr());
   return cuda_fail(cudaGetLastError(), "score_stream_kernel");
 }
 
@@ -760,16 +916,28 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
   sc.qo = a.p->query_offsets;
   sc.q_pos = a.p->q_pos;
   sc.S = a.p->num_seqs;
+  const CandLayout cl = cand_layout(a.grid, a.subcap);
+  uint8_t* base = reinterpret_cast<uint8_t*>(a.cand);
+  Lists main_ls, fix_ls;
+  main_ls.cand = reinterpret_cast<uint2*>(base);
+  main_ls.cnt = reinterpret_cast<int*>(base + cl.main_lists);
+  main_ls.rows_cap = cl.rows_main;
+  main_ls.slots = kMaxG;
+  fix_ls.cand = reinterpret_cast<uint2*>(base + cl.main_lists + cl.main_counts);
+  fix_ls.cnt = reinterpret_cast<int*>(base + cl.main_lists + cl.main_counts + cl.fix_lists);
+  fix_ls.rows_cap = cl.rows_full;
+  fix_ls.slots = 1;
   cudaError_t e = cudaMemsetAsync(a.fail_count, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "reset failure count");
-  int rc = launch_one<MH>(a, kmap, qmap, sc, st);
+  int rc = launch_one<MH>(a, kmap, qmap, sc, main_ls, st);
   if (rc) return rc;
-  // Queries whose probe threshold did not verify: rescan without a probe.
+  // Queries whose probe threshold did not verify: rescan without a probe,
+  // one query per group, with lists that hold every key.
   Sched fx = sc;
   fx.fail_in = a.fail_list;
   fx.fail_out = nullptr;
   fx.count = a.fail_count;
-  return launch_one<MH>(a, kmap, qmap, fx, st);
+  return launch_one<MH>(a, kmap, qmap, fx, fix_ls, st);
 }
 
 }  // namespace
@@ -782,8 +950,8 @@ int64_t stream_subcap(int max_seq_len) {
 }
 
 size_t stream_cand_bytes(int grid, int64_t subcap) {
-  // lists [grid][kMaxG][subcap rows][128], then counts [grid][kMaxG][128]
-  return (size_t)grid * kMaxG * 128 * ((size_t)subcap * sizeof(uint2) + sizeof(int));
+  const CandLayout c = cand_layout(grid, subcap);
+  return c.main_lists + c.main_counts + c.fix_lists + c.fix_counts;
 }
 
 int launch_score_stream(const StreamArgs& a, cudaStream_t st) {
