@@ -270,7 +270,7 @@ StreamPlan stream_plan(const misa_problem_t* p, int m, int k, bool want_rows) {
   sp.grid = sms < sp.max_groups ? sms : sp.max_groups;
   sp.cap = stream_subcap(p->max_seq_len);
   sp.bytes = groups_bytes(T, p->num_seqs) + fail_bytes(T) +
-             align_up(stream_cand_bytes(sp.grid, sp.cap));
+             align_up(stream_cand_bytes(sp.grid, sp.cap, m));
   sp.use = true;
   return sp;
 }

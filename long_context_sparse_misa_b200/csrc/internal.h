@@ -121,7 +121,7 @@ struct StreamArgs {
   int max_groups;
   int grid;               // persistent CTAs (<= number of SMs)
   int k;
-  uint2* cand;            // stream_cand_bytes(grid, subcap): candidate lists and counts
+  uint2* cand;            // stream_cand_bytes(grid, subcap, m): candidate lists and counts
   int64_t subcap;         // stream_subcap(max_seq_len): rows of each list
   int32_t* idx;
   float* val;
@@ -130,7 +130,7 @@ struct StreamArgs {
 };
 int launch_score_stream(const StreamArgs& a, cudaStream_t st);
 int stream_group_size(int m);
-size_t stream_cand_bytes(int grid, int64_t subcap);
+size_t stream_cand_bytes(int grid, int64_t subcap, int m);
 int64_t stream_subcap(int max_seq_len);
 int score_group_size(int m);
 

@@ -66,7 +66,12 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kSelWarps = 2;
 // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue, warps 18..19 selectors
 constexpr int kThreads = 64 + kEpiThreads + 32 * kSelWarps;
-constexpr int kRowsCap = 128;                    // rows per candidate list (main pass)
+// Rows per main-pass candidate list: about 21 are used at 128K with the
+// probe threshold; a query whose threshold is no filter (short prefixes) or
+// that runs past 128 rows goes to the rescan launch, whose lists hold every
+// key.  (Letting such queries fill full-length lists makes their exact
+// selection, one warp per query, far slower than the rescan.)
+constexpr int kRowsCap = 128;
 constexpr int kParts = kEpiWarps / 4;            // column parts per TMEM lane quarter
 constexpr int kColsPerWarp = kN / kParts;
 constexpr int kQHalfBytes = kN * 128;            // 32 KB per 64-dim half
@@ -872,7 +877,7 @@ __global__ void __maxnreg__(96)
 }
 
 // Candidate storage (one workspace region, 256-byte aligned parts): the main
-// pass's lists [grid][2][kMaxG][rows_main][128] and counts, then the rescan's
+// pass's lists [grid][2][G][rows_main][128] and counts, then the rescan's
 // lists [grid][2][1][rows_full][128] and counts.
 struct CandLayout {
   int rows_main, rows_full;
@@ -881,12 +886,12 @@ struct CandLayout {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-CandLayout cand_layout(int grid, int64_t rows_full) {
+CandLayout cand_layout(int grid, int64_t rows_full, int G) {
   CandLayout c;
   c.rows_full = (int)rows_full;
-  c.rows_main = rows_full < kRowsCap ? (int)rows_full : kRowsCap;
-  c.main_lists = align256((size_t)grid * 2 * kMaxG * c.rows_main * 128 * sizeof(uint2));
-  c.main_counts = align256((size_t)grid * 2 * kMaxG * 128 * sizeof(int));
+  c.rows_main = (int)(rows_full < kRowsCap ? rows_full : kRowsCap);
+  c.main_lists = align256((size_t)grid * 2 * G * c.rows_main * 128 * sizeof(uint2));
+  c.main_counts = align256((size_t)grid * 2 * G * 128 * sizeof(int));
   c.fix_lists = align256((size_t)grid * 2 * c.rows_full * 128 * sizeof(uint2));
   c.fix_counts = align256((size_t)grid * 2 * 128 * sizeof(int));
   return c;
@@ -916,13 +921,13 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
   sc.qo = a.p->query_offsets;
   sc.q_pos = a.p->q_pos;
   sc.S = a.p->num_seqs;
-  const CandLayout cl = cand_layout(a.grid, a.subcap);
+  const CandLayout cl = cand_layout(a.grid, a.subcap, kN / MH);
   uint8_t* base = reinterpret_cast<uint8_t*>(a.cand);
   Lists main_ls, fix_ls;
   main_ls.cand = reinterpret_cast<uint2*>(base);
   main_ls.cnt = reinterpret_cast<int*>(base + cl.main_lists);
   main_ls.rows_cap = cl.rows_main;
-  main_ls.slots = kMaxG;
+  main_ls.slots = kN / MH;
   fix_ls.cand = reinterpret_cast<uint2*>(base + cl.main_lists + cl.main_counts);
   fix_ls.cnt = reinterpret_cast<int*>(base + cl.main_lists + cl.main_counts + cl.fix_lists);
   fix_ls.rows_cap = cl.rows_full;
@@ -949,8 +954,8 @@ int64_t stream_subcap(int max_seq_len) {
   return ((int64_t)max_seq_len + kTileKeys - 1) / kTileKeys;
 }
 
-size_t stream_cand_bytes(int grid, int64_t subcap) {
-  const CandLayout c = cand_layout(grid, subcap);
+size_t stream_cand_bytes(int grid, int64_t subcap, int m) {
+  const CandLayout c = cand_layout(grid, subcap, kN / m);
   return c.main_lists + c.main_counts + c.fix_lists + c.fix_counts;
 }
 
