@@ -22,7 +22,7 @@
 // tile: tcgen05.ld of 32 columns, wait, then per key and query
 // I = sum_j w_j ReLU(acc_j) (the TMEM buffer is released after the warp's
 // last load), the causal mask, and the streaming selection:
-//   * probe: a group first scores every 8th tile of its prefix and keeps a
+//   * probe: a group first scores every 24th tile of its prefix and keeps a
 //     256-bin histogram per query (1/32-octave bins of the order-preserving
 //     score key, from 7 octaves below the first scored tile's maximum to one
 //     above; scores outside fall into the end bins, which can only lower the
@@ -83,8 +83,8 @@ constexpr int kHistWords = kBins / 2;            // two 16-bit bin counts per wo
 constexpr int kBinShift = 18;                    // 14-bit score key prefix: 1/32 octave
 constexpr int kHeadroom = 224;                   // bins below the first tile's maximum
 constexpr int kSelBins = 256;
-constexpr int kProbeStride = 8;                  // probe every 8th tile ...
-constexpr int kProbeOff = 4;                     // ... starting at tile 4
+constexpr int kProbeStride = 24;                 // probe every 24th tile ...
+constexpr int kProbeOff = 12;                    // ... starting at tile 12
 constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
 
 static_assert(kSelBins >= kBins, "final-select histogram");

@@ -152,9 +152,10 @@ def test_stream_exact_ties_resolve_to_lower_index():
 
 
 def test_stream_probe_overestimate_goes_through_fixup():
-    # Only the probed tiles (every 8th, from tile 4) hold high scores, and only
-    # on half their keys: the sampled threshold then admits fewer than k keys,
-    # the check fails and those queries are rescanned without a probe.
+    # The probed tiles (every 24th, from tile 12) all lie among the tiles that
+    # hold high scores (every 8th, from tile 4), on half their keys: the
+    # sampled threshold then admits fewer than k keys, the check fails and
+    # those queries are rescanned without a probe.
     L, H, d = 10000, 8, 128
     wl = make_workload(seq_lens=[L], queries="all", H=H, B=64, m=8, k=2048, seed=6,
                        needles=False)
