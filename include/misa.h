@@ -130,8 +130,10 @@ int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const
  *   - Calls on one device must not overlap in execution: they share the
  *     array and race on it.  Issue them on one stream, or order them.
  *   - MISA_ERR_UNSUPPORTED when the problem needs more than 4 MiB of router
- *     scratch (the message gives both sizes); MISA_ERR_INVALID_ARG while
- *     tracing is on for the calling thread. */
+ *     scratch (the message gives both sizes): decode batches fit; prefill
+ *     fits up to about 7K keys, since the tensor-core router keeps a 512-byte
+ *     running block mean per key.  MISA_ERR_INVALID_ARG while tracing is on
+ *     for the calling thread. */
 int misa_route_static(const misa_problem_t* p, const uint16_t* q, const float* w,
                       const uint16_t* K, const float* Kbar, int32_t m, int32_t* heads,
                       uint16_t* q_r, float* w_r, float* router_scores, misa_stream_t stream);

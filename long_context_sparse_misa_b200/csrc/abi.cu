@@ -247,7 +247,7 @@ size_t route_bytes(const misa_problem_t* p) {
 }
 
 size_t route_tc_bytes(const misa_problem_t* p) {
-  return groups_bytes(p->num_queries, p->num_seqs) + align_up(route_tc_split_bytes(p->total_blocks));
+  return groups_bytes(p->num_queries, p->num_seqs) + align_up(route_tc_split_bytes(*p));
 }
 
 // Streaming (fused top-k) scorer: used when every query scores its whole

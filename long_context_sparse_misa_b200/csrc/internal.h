@@ -80,11 +80,12 @@ struct RouteTcArgs {
   const int4* groups;     // route_tc_group_size(H) queries per group
   const int* group_count;
   int max_groups;
-  void* split;            // route_tc_split_bytes(total_blocks) of workspace
+  void* split;            // route_tc_split_bytes(p) of workspace
+  float* Pm;              // set by launch_route_tc (inside split)
 };
 int launch_route_tc(const RouteTcArgs& a, cudaStream_t st);
 int route_tc_group_size(int H);
-size_t route_tc_split_bytes(int64_t total_blocks);
+size_t route_tc_split_bytes(const misa_problem_t& p);
 
 // ---- score.cu
 // I[(t - q_lo) * ld + s] = sum_{j<m} wsel[t,j] ReLU(qsel[t,j] . K[key(t,s)]) for the

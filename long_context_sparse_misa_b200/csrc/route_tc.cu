@@ -17,7 +17,10 @@
 // accumulated into the same fp32 accumulator, which keeps ~16 mantissa bits
 // of the pooled keys.  Epilogue warps own one row of each accumulator per
 // lane, so the block-axis ReLU-sum is inside the thread; an accumulator is
-// released as soon as it is copied to registers.
+// released as soon as it is copied to registers.  The causal partial block
+// of every key position (the running mean of its block up to that key) is
+// computed beforehand by one warp per pooled block, so each query only
+// reads its row.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,13 +36,12 @@ constexpr int kHalfBytes = kStageBytes / 2;
 constexpr int kQHalfBytes = kRows * 128;              // 64 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kMaxG = 16;                             // queries per group
-constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kMaxG * kD * 4 /*P*/ +
-                           kRows * 4 /*r*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kRows * 4 /*r*/ +
+                           kMaxG * 4 * 2 + 16 * 8 + 16;
 
 struct Smem {
   uint8_t* q;
   uint8_t* k;
-  float* P;   // [kMaxG][128] causal partial-block means
   float* r;   // [kRows] router scores of the group
   int* pos;
   int* flags;
@@ -59,8 +61,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.q = p;
   s.k = p + kQBytes;
-  s.P = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
-  s.r = s.P + kMaxG * kD;
+  s.r = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
   s.pos = reinterpret_cast<int*>(s.r + kRows);
   s.flags = s.pos + kMaxG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
@@ -86,6 +87,41 @@ __global__ void split_kbar_kernel(const float* __restrict__ Kbar, int64_t n,
   lo[i] = __float2bfloat16_rn(x - __bfloat162float(h));
 }
 
+// Running block means of the keys: Pm[key] = mean of the keys from the start
+// of key's pooled block up to key, summed in key order (fp32).  One warp per
+// pooled block; each lane owns 4 of the 128 dims; 8 keys' loads in flight.
+__global__ void __launch_bounds__(256)
+    prefix_means_kernel(const uint16_t* __restrict__ K, const int64_t* __restrict__ ko,
+                        const int64_t* __restrict__ bo, int S, int B, int64_t total_blocks,
+                        float* __restrict__ Pm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= total_blocks) return;
+  const int s = upper_segment<int64_t>(bo, S, row);
+  const int64_t k0 = ko[s] + (row - bo[s]) * B;
+  const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
+  const uint2* src = reinterpret_cast<const uint2*>(K) + lane;
+  float4* dst = reinterpret_cast<float4*>(Pm) + lane;
+  float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+  for (int64_t kb = k0; kb < k1; kb += 8) {
+    uint2 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = kb + u < k1 ? __ldg(src + (kb + u) * (kD / 4)) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t key = kb + u;
+      if (key >= k1) break;
+      r0 += __uint_as_float(v[u].x << 16);
+      r1 += __uint_as_float(v[u].x & 0xFFFF0000u);
+      r2 += __uint_as_float(v[u].y << 16);
+      r3 += __uint_as_float(v[u].y & 0xFFFF0000u);
+      const float cnt = (float)(key - k0 + 1);
+      dst[key * (kD / 4)] = make_float4(r0 / cnt, r1 / cnt, r2 / cnt, r3 / cnt);
+    }
+  }
+}
+
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -94,7 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float* __restrict__ w, const uint16_t* __restrict__ K,
                     const int64_t* __restrict__ ko, const int64_t* __restrict__ bo,
                     const int32_t* __restrict__ q_pos, const int4* __restrict__ groups,
-                    const int* __restrict__ group_count, int B, int m,
+                    const int* __restrict__ group_count, const float* __restrict__ Pm, int B,
+                    int m,
                     int32_t* __restrict__ heads, uint16_t* __restrict__ q_r,
                     float* __restrict__ w_r, float* __restrict__ router_scores,
                     uint32_t* status) {
@@ -227,48 +264,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
 
-    // Causal partial-block means P[qi] (mean of keys floor((t+1)/B)*B .. t),
-    // thread = dimension; overlaps the first chunks' MMAs.
-    {
-      const int d = et;
-      const uint16_t* Kseq = K + ko[seq] * kD + d;
-      bool consec = true;
-      for (int qi = 1; qi < nq; ++qi) consec &= (s.pos[qi] == s.pos[0] + qi) && s.pos[qi] >= 0;
-      consec &= s.pos[0] >= 0;
-      if (consec) {
-        // Running block sums in key order; 16 loads in flight per thread.
-        const int p0 = s.pos[0], p1 = s.pos[nq - 1];
-        const int k0 = (p0 / B) * B;
-        float run = 0.f;
-        for (int kb = k0; kb <= p1; kb += 16) {
-          float x[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            x[u] = kb + u <= p1 ? bf16_bits_to_float(Kseq[(int64_t)(kb + u) * kD]) : 0.f;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int key = kb + u;
-            if (key > p1) break;
-            if (key % B == 0) run = 0.f;
-            run += x[u];
-            if (key >= p0) {
-              const int cntv = key - (key / B) * B + 1;
-              s.P[(key - p0) * kD + d] = run / (float)cntv;
-            }
-          }
-        }
-      } else {
-        for (int qi = 0; qi < nq; ++qi) {
-          const int p = s.pos[qi];
-          if (p < 0 || (p + 1) % B == 0) continue;
-          const int f = (p + 1) / B * B;
-          float run = 0.f;
-          for (int key = f; key <= p; ++key) run += bf16_bits_to_float(Kseq[(int64_t)key * kD]);
-          s.P[qi * kD + d] = run / (float)(p + 1 - f);
-        }
-      }
-    }
-
     // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
     // of every accumulator.
     float acc[NSUB];
@@ -333,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float total = acc[sub];
           if ((p + 1) % B != 0) {
             const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)(qb + qi) * H + h) * kD);
-            const float* Pq = s.P + qi * kD;
+            const float* Pq = Pm + (ko[seq] + p) * kD;  // running block mean at p
             float dp = 0.f;
 #pragma unroll
             for (int i = 0; i < kD / 8; ++i) {
@@ -416,7 +411,7 @@ int launch_h(const RouteTcArgs& a, const CUtensorMap& qmap, const CUtensorMap& h
   ProfScope ps("route", st);
   kern<<<a.max_groups, kThreads, kSmemBytes, st>>>(
       qmap, himap, lomap, a.q, a.w, a.K, a.p->key_offsets, a.p->block_offsets, a.p->q_pos,
-      a.groups, a.group_count, a.p->block, a.m, a.heads, a.q_r, a.w_r, a.router_scores,
+      a.groups, a.group_count, a.Pm, a.p->block, a.m, a.heads, a.q_r, a.w_r, a.router_scores,
       status_ptr());
   return cuda_fail(cudaGetLastError(), "route_tc_kernel");
 }
@@ -428,8 +423,10 @@ int route_tc_group_size(int H) {
   return g < kMaxG ? g : kMaxG;
 }
 
-size_t route_tc_split_bytes(int64_t total_blocks) {
-  return (size_t)total_blocks * kD * 2 * 2;  // hi + lo bf16
+size_t route_tc_split_bytes(const misa_problem_t& p) {
+  // hi + lo bf16 copies of Kbar, then the running block means (fp32 per key)
+  const size_t split = ((size_t)p.total_blocks * kD * 2 * 2 + 255) & ~size_t(255);
+  return split + (size_t)p.total_keys * kD * 4;
 }
 
 int launch_route_tc(const RouteTcArgs& a, cudaStream_t st) {
@@ -438,6 +435,16 @@ int launch_route_tc(const RouteTcArgs& a, cudaStream_t st) {
   const int64_t n = p.total_blocks * kD;
   __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.split);
   __nv_bfloat16* lo = hi + n;
+  RouteTcArgs b = a;
+  b.Pm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.split) +
+                                  (((size_t)n * 2 * 2 + 255) & ~size_t(255)));
+  if (p.total_blocks > 0) {
+    ProfScope ps("route_means", st);
+    prefix_means_kernel<<<(unsigned)((p.total_blocks + 7) / 8), 256, 0, st>>>(
+        a.K, p.key_offsets, p.block_offsets, p.num_seqs, p.block, p.total_blocks, b.Pm);
+    int rc = cuda_fail(cudaGetLastError(), "prefix_means_kernel");
+    if (rc) return rc;
+  }
   if (n > 0) {
     ProfScope ps("route_split", st);
     split_kbar_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.Kbar, n, hi, lo);
@@ -450,10 +457,10 @@ int launch_route_tc(const RouteTcArgs& a, cudaStream_t st) {
   if ((rc = make_kmajor_map(&himap, hi, p.total_blocks, kChunk))) return rc;
   if ((rc = make_kmajor_map(&lomap, lo, p.total_blocks, kChunk))) return rc;
   switch (p.num_heads) {
-    case 8: return launch_h<8>(a, qmap, himap, lomap, st);
-    case 16: return launch_h<16>(a, qmap, himap, lomap, st);
-    case 32: return launch_h<32>(a, qmap, himap, lomap, st);
-    case 64: return launch_h<64>(a, qmap, himap, lomap, st);
+    case 8: return launch_h<8>(b, qmap, himap, lomap, st);
+    case 16: return launch_h<16>(b, qmap, himap, lomap, st);
+    case 32: return launch_h<32>(b, qmap, himap, lomap, st);
+    case 64: return launch_h<64>(b, qmap, himap, lomap, st);
     default:
       set_error("tensor-core router needs H in {8,16,32,64}, got %d", p.num_heads);
       return MISA_ERR_UNSUPPORTED;
