@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--max-queries", type=int, default=0,
                     help="keep only the last N queries (small captures for ncu)")
+    ap.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
+                    help="replay each step as one CUDA graph (auto: decode workloads)")
     return ap.parse_args()
 
 
@@ -298,7 +300,19 @@ def run_ours(args):
     q = torch.from_numpy(wl.q_bits).to(dev)
     w = torch.from_numpy(wl.w).to(dev)
     ix = misa.Indexer(prob, m=wl.m, k=wl.k, k_cand=wl.k_cand, device=dev)
-    run = (lambda: ix.hier(q, w, K)) if hier else (lambda: ix.misa(q, w, K))
+    from misa_synth import CONFIGS
+    decode = CONFIGS[cfg]["queries"] != "all"
+    use_graph = args.graph == "on" or (args.graph == "auto" and decode)
+    # Decode step: the keys before this step's queries were pooled by earlier
+    # steps, so only the blocks holding the new keys are re-pooled.
+    pool_from = None
+    if decode:
+        q_per_seq = np.diff(wl.query_offsets)
+        pool_from = torch.tensor(wl.seq_lens - q_per_seq, dtype=torch.int32, device=dev)
+        misa.pool_keys(prob, K, ix.Kbar)
+    run = ((lambda: ix.hier(q, w, K, pool_from=pool_from)) if hier
+           else (lambda: ix.misa(q, w, K, pool_from=pool_from)))
+    eager_run = run
     small_inputs = wl.q_bits.nbytes + wl.K_bits.nbytes < 2 * 126e6
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small_inputs else None
 
@@ -313,12 +327,29 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {code} ({bits}) after warm-up")
 
+    def capture(fn):
+        """One step as a CUDA graph (all of the library's launches)."""
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    graph = capture(eager_run) if use_graph else None
+    if graph is not None:
+        run = graph.replay
+
     # ---- timed region (device time, CUDA events, max over ranks)
     props = torch.cuda.get_device_properties(dev)
     clocks = Clocks(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
     torch.cuda.synchronize()
     barrier(world)
-    misa.profile_enable(True)
+    misa.profile_enable(graph is None)
     clocks.start()
     # Each step is bracketed by its own events; the L2 flush (small inputs
     # only) runs between steps, outside the timed intervals.
@@ -335,7 +366,22 @@ def run_ours(args):
     prof = misa.profile_collect()
     misa.profile_enable(False)
     barrier(world)
-    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs), world)
+    step_ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+    ms = max_over_ranks(sum(step_ms), world)
+    p50 = max_over_ranks(step_ms[len(step_ms) // 2], world)
+    p90 = max_over_ranks(step_ms[min(len(step_ms) - 1, (9 * len(step_ms)) // 10)], world)
+    if graph is not None:
+        # Per-kernel times come from the same step launched eagerly (a graph
+        # replay has no per-launch events), outside the timed region.
+        torch.cuda.synchronize()
+        misa.profile_enable(True)
+        for _ in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            eager_run()
+        torch.cuda.synchronize()
+        prof = misa.profile_collect()
+        misa.profile_enable(False)
     code, bits = misa.stream_status()
     if code != 0:
         raise RuntimeError(f"device status {code} ({bits}) in the timed region")
@@ -348,20 +394,37 @@ def run_ours(args):
     kname = "score"
     k_ms, k_launch = prof.get(kname, (float("nan"), 0))
     streamed = "topk" not in prof
-    flops = 2.0 * wl.m * wl.d * pairs * args.steps
-    achieved = flops / (k_ms / 1e3) / 1e12
+    launches_per_step = k_launch / args.steps
     tpp = traffic_per_pair("score_stream" if streamed else "score",
                            workload_config(wl, cfg)["workload"])
-    launches_per_step = k_launch / args.steps
-    roofline = {"kernel": ("score_stream_kernel (tcgen05 routed scoring, top-k in the epilogue)"
-                           if streamed else "score_kernel (tcgen05 routed scoring)"),
-                "bound": "tensor",
-                "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_sustained"],
-                "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
-                "algorithmic_flops_per_launch": 2.0 * wl.m * wl.d * pairs / max(launches_per_step, 1),
-                "launches_per_step": launches_per_step,
-                "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
+    if streamed:
+        # prefill: a dense contraction, 2*m*d flops per scored pair
+        flops = 2.0 * wl.m * wl.d * pairs * args.steps
+        achieved = flops / (k_ms / 1e3) / 1e12
+        roofline = {"kernel": "score_stream_kernel (tcgen05 routed scoring, top-k in the epilogue)",
+                    "bound": "tensor",
+                    "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_sustained"],
+                    "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                    "algorithmic_flops_per_launch": 2.0 * wl.m * wl.d * pairs / max(launches_per_step, 1)}
+    else:
+        # decode: HBM-bound; each query group streams its prefix of K once
+        # (256 B per key) and writes its fp32 score rows (4 B per pair)
+        G = 256 // wl.m
+        kbytes = 0
+        for s_ in range(len(wl.seq_lens)):
+            pos = wl.q_pos[wl.query_offsets[s_]:wl.query_offsets[s_ + 1]]
+            for g0 in range(0, len(pos), G):
+                kbytes += (int(pos[g0:g0 + G].max()) + 1) * 256
+        abytes = kbytes + 4 * pairs
+        achieved = abytes * args.steps / (k_ms / 1e3) / 1e9
+        roofline = {"kernel": "score_kernel (tcgen05 routed scoring, score rows)",
+                    "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "peak_source": f"hbm_gbs ({peaks['source']})",
+                    "algorithmic_bytes_per_launch": abytes / max(launches_per_step, 1)}
+    roofline |= {"launches_per_step": launches_per_step,
+                 "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
     kernels = {n: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps,
                    "share": t / max(sum(v[0] for v in prof.values()), 1e-9)}
                for n, (t, c) in prof.items()}
@@ -373,8 +436,12 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 q,k with 1% planted needles; "
                     "w ~ N(0,1)/sqrt(H) fp32)",
             "config": workload_config(wl, cfg) | {"parallelism": f"independent problem per GPU x{world}"},
-            "latency_ms": ms_step, "roofline": roofline, "kernels": kernels,
+            "latency_ms": ms_step, "step_ms_p50": p50, "step_ms_p90": p90,
+            "cuda_graph": graph is not None,
+            "roofline": roofline, "kernels": kernels,
             "gpu_launches": gpu_launches, "clocks": clk}
+    if decode:
+        line["config"]["decode_step"] = "pooled keys of earlier blocks kept; blocks with new keys re-pooled"
 
     # ---- dense DSA indexer on the same inputs (the in-run comparison)
     if not args.no_dense:
@@ -384,20 +451,31 @@ def run_ours(args):
                 flush.fill_(1)
             ix.dense(q, w, K)
         torch.cuda.synchronize()
+        dense_run = lambda: ix.dense(q, w, K)
+        dgraph = capture(dense_run) if use_graph else None
+        if dgraph is not None:
+            dense_run = dgraph.replay
         barrier(world)
-        misa.profile_enable(True)
+        misa.profile_enable(dgraph is None)
         devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(dense_steps)]
         for e0, e1 in devs:
             if flush is not None:
                 flush.fill_(1)
             e0.record()
-            ix.dense(q, w, K)
+            dense_run()
             e1.record()
         torch.cuda.synchronize()
         dprof = misa.profile_collect()
         misa.profile_enable(False)
         dms = max_over_ranks(sum(a.elapsed_time(b) for a, b in devs), world) / dense_steps
+        if dgraph is not None:
+            misa.profile_enable(True)
+            for _ in range(dense_steps):
+                ix.dense(q, w, K)
+            torch.cuda.synchronize()
+            dprof = misa.profile_collect()
+            misa.profile_enable(False)
         d_k_ms = dprof.get("score", (float("nan"), 0))[0] / dense_steps
         d_flops = 2.0 * wl.H * wl.d * pairs
         line["dense_dsa"] = {"ms_per_step": dms, "value": job_throughput(pairs, world, dms),
@@ -417,7 +495,7 @@ def run_ours(args):
             K.copy_(K_h, non_blocking=True)
             q.copy_(q_h, non_blocking=True)
             w.copy_(w_h, non_blocking=True)
-            run()
+            eager_run()  # the public API calls, launched one by one
             idx_h.copy_(ix.idx, non_blocking=True)
             val_h.copy_(ix.val, non_blocking=True)
 

@@ -103,6 +103,18 @@ int misa_block_offsets(const int64_t* key_offsets, int32_t num_seqs, int32_t blo
  *   K    [total_keys, 128] bf16;  Kbar [total_blocks, 128] fp32 (written). */
 int misa_pool_keys(const misa_problem_t* p, const uint16_t* K, float* Kbar, misa_stream_t stream);
 
+/* Step 1, incremental (decode): re-pools only the blocks of each sequence s
+ * that hold keys at positions >= from_pos[s] (e.g. the keys appended since
+ * Kbar was last computed); every other row of Kbar is left unchanged, so
+ * Kbar must already hold the pooled means of the earlier blocks.  Same
+ * arithmetic as misa_pool_keys, so the updated rows are bit-identical to a
+ * full re-pooling.
+ *   from_pos [S] int32 device array; a value <= 0 re-pools the whole
+ *   sequence, a value >= its length leaves it unchanged.  One CTA per
+ *   sequence. */
+int misa_pool_keys_from(const misa_problem_t* p, const uint16_t* K, float* Kbar,
+                        const int32_t* from_pos, misa_stream_t stream);
+
 /* Step 2 -- block-pooled router (same passage: per-head affinities on the
  * pooled keys, aggregated into one importance score per head, top-h heads).
  *     r[t,h] = w[t,h] * sum_{b < M_t} ReLU(q[t,h] . Kbar_t[b]),  M_t = ceil((t+1)/B)

@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "LIB_PATH", "lib", "MisaError", "Problem", "workspace_size", "block_offsets", "pool_keys",
-    "route", "score_topk", "hier_rerank", "dsa_index_dense", "stream_status",
+    "route", "pool_keys_from", "score_topk", "hier_rerank", "dsa_index_dense", "stream_status",
     "selftest_timeout", "route_static", "EXPORTED", "Indexer", "profile_enable", "profile_collect",
 ]
 
@@ -26,7 +26,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmisa.so"
 
 # Every symbol include/misa.h declares.
 EXPORTED = (
-    "misa_workspace_size", "misa_block_offsets", "misa_pool_keys", "misa_route",
+    "misa_workspace_size", "misa_block_offsets", "misa_pool_keys", "misa_pool_keys_from",
+    "misa_route",
     "misa_route_static", "misa_score_topk", "misa_hier_rerank", "dsa_index_dense", "misa_stream_status",
     "misa_selftest_timeout", "misa_profile_enable", "misa_profile_collect",
     "misa_last_error_string",
@@ -55,6 +56,7 @@ _sig = {
     "misa_workspace_size": (_c_sz, [_PP, _c_i32, _c_i32, _c_i32]),
     "misa_block_offsets": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p]),
     "misa_pool_keys": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p]),
+    "misa_pool_keys_from": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p]),
     "misa_route": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p,
                                   _c_p, _c_sz, _c_p]),
     "misa_route_static": (ctypes.c_int, [_PP, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p,
@@ -170,6 +172,11 @@ def pool_keys(prob: Problem, K, Kbar, stream=None) -> None:
     _check(lib.misa_pool_keys(prob.ref, _ptr(K), _ptr(Kbar), _stream(stream)), "misa_pool_keys")
 
 
+def pool_keys_from(prob: Problem, K, Kbar, from_pos, stream=None) -> None:
+    _check(lib.misa_pool_keys_from(prob.ref, _ptr(K), _ptr(Kbar), _ptr(from_pos),
+                                   _stream(stream)), "misa_pool_keys_from")
+
+
 def route(prob: Problem, q, w, K, Kbar, m: int, heads, q_r, w_r, router_scores, ws,
           stream=None) -> None:
     _check(lib.misa_route(prob.ref, _ptr(q), _ptr(w), _ptr(K), _ptr(Kbar), m, _ptr(heads),
@@ -268,19 +275,24 @@ class Indexer:
             self.cand = torch.empty((T, k_cand), dtype=torch.int32, device=dev)
             self.cand_val = torch.empty((T, k_cand), dtype=torch.float32, device=dev)
 
-    def pool_route(self, q, w, K, stream=None):
-        pool_keys(self.prob, K, self.Kbar, stream)
+    def pool_route(self, q, w, K, stream=None, pool_from=None):
+        """pool_from: None re-pools every block; else an int32 device tensor
+        [S] of first new key positions (Kbar must hold the earlier blocks)."""
+        if pool_from is None:
+            pool_keys(self.prob, K, self.Kbar, stream)
+        else:
+            pool_keys_from(self.prob, K, self.Kbar, pool_from, stream)
         route(self.prob, q, w, K, self.Kbar, self.m, self.heads, self.q_r, self.w_r, self.r,
               self.ws, stream)
 
-    def misa(self, q, w, K, stream=None, scores_dbg=None):
-        self.pool_route(q, w, K, stream)
+    def misa(self, q, w, K, stream=None, scores_dbg=None, pool_from=None):
+        self.pool_route(q, w, K, stream, pool_from)
         score_topk(self.prob, self.q_r, self.w_r, self.m, K, self.k, self.idx, self.val,
                    self.ws, scores_dbg, stream)
         return self.idx, self.val
 
-    def hier(self, q, w, K, stream=None):
-        self.pool_route(q, w, K, stream)
+    def hier(self, q, w, K, stream=None, pool_from=None):
+        self.pool_route(q, w, K, stream, pool_from)
         score_topk(self.prob, self.q_r, self.w_r, self.m, K, self.k_cand, self.cand,
                    self.cand_val, self.ws, None, stream)
         hier_rerank(self.prob, q, w, K, self.cand, self.k_cand, self.k, self.idx, self.val,

@@ -416,6 +416,17 @@ int misa_pool_keys(const misa_problem_t* p, const uint16_t* K, float* Kbar,
   return launch_pool(*p, K, Kbar, static_cast<cudaStream_t>(stream));
 }
 
+int misa_pool_keys_from(const misa_problem_t* p, const uint16_t* K, float* Kbar,
+                        const int32_t* from_pos, misa_stream_t stream) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (p->total_blocks == 0) return MISA_OK;
+  if ((rc = check_ptr(K, 16, "K")) || (rc = check_ptr(Kbar, 16, "Kbar")) ||
+      (rc = check_ptr(from_pos, 4, "from_pos")))
+    return rc;
+  return launch_pool_from(*p, K, Kbar, from_pos, static_cast<cudaStream_t>(stream));
+}
+
 int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const uint16_t* K,
                const float* Kbar, int32_t m, int32_t* heads, uint16_t* q_r, float* w_r,
                float* router_scores, void* ws, size_t ws_bytes, misa_stream_t stream) {

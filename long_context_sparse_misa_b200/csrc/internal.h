@@ -53,6 +53,9 @@ int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* bloc
 int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
                        int* count, cudaStream_t st);
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st);
+// Re-pool only the blocks of each sequence s that hold keys >= from_pos[s].
+int launch_pool_from(const misa_problem_t& p, const uint16_t* K, float* Kbar,
+                     const int32_t* from_pos, cudaStream_t st);
 
 // ---- route.cu
 int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, const uint16_t* K,

@@ -146,22 +146,10 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 v) {
   acc[7] += (double)__uint_as_float(v.w & 0xFFFF0000u);
 }
 
-__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ K,
-                                                   const int64_t* __restrict__ ko,
-                                                   const int64_t* __restrict__ bo, int S, int B,
-                                                   int64_t total_blocks, int64_t total_keys,
-                                                   float* __restrict__ Kbar, uint32_t* status) {
+// Mean of the keys of pooled row `row` of sequence s (block b), by one warp.
+__device__ __forceinline__ void pool_row(const uint16_t* __restrict__ K, int64_t k0, int64_t k1,
+                                         int64_t row, float* __restrict__ Kbar) {
   const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= total_blocks) return;
-  const int s = upper_segment<int64_t>(bo, S, row);
-  const int64_t b = row - bo[s];
-  const int64_t k0 = ko[s] + b * B;
-  const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
-  if (k0 < 0 || k1 > total_keys || k1 <= k0) {
-    if (lane == 0) set_status(status, MISA_STATUS_BOUNDS);
-    return;
-  }
   constexpr int kRow16 = kD / 8;  // 16-byte chunks per key
   const int half = lane >> 4, hl = lane & 15;
   double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
@@ -195,6 +183,54 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   }
 }
 
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ K,
+                                                   const int64_t* __restrict__ ko,
+                                                   const int64_t* __restrict__ bo, int S, int B,
+                                                   int64_t total_blocks, int64_t total_keys,
+                                                   float* __restrict__ Kbar, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= total_blocks) return;
+  const int s = upper_segment<int64_t>(bo, S, row);
+  const int64_t b = row - bo[s];
+  const int64_t k0 = ko[s] + b * B;
+  const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
+  if (k0 < 0 || k1 > total_keys || k1 <= k0) {
+    if (lane == 0) set_status(status, MISA_STATUS_BOUNDS);
+    return;
+  }
+  pool_row(K, k0, k1, row, Kbar);
+}
+
+// Incremental form: one CTA per sequence re-pools only the blocks that hold
+// keys at or after from_pos[s] (the keys appended since the last pooling);
+// the other rows of Kbar are left as they are.  Warps take the blocks
+// round-robin.
+__global__ void __launch_bounds__(256) pool_from_kernel(const uint16_t* __restrict__ K,
+                                                        const int64_t* __restrict__ ko,
+                                                        const int64_t* __restrict__ bo, int B,
+                                                        const int32_t* __restrict__ from_pos,
+                                                        float* __restrict__ Kbar,
+                                                        uint32_t* status) {
+  const int s = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int64_t L = ko[s + 1] - ko[s];
+  const int64_t nblk = bo[s + 1] - bo[s];
+  int64_t f = from_pos[s];
+  if (f < 0) f = 0;
+  if (f >= L) return;  // nothing new in this sequence
+  if (nblk != (L + B - 1) / B) {
+    if (threadIdx.x == 0) set_status(status, MISA_STATUS_BOUNDS);
+    return;
+  }
+  for (int64_t b = f / B + warp; b < nblk; b += nw) {
+    const int64_t k0 = ko[s] + b * B;
+    const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
+    pool_row(K, k0, k1, bo[s] + b, Kbar);
+  }
+  (void)lane;
+}
+
 }  // namespace
 
 int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* block_offsets,
@@ -217,6 +253,14 @@ int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4*
       p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo, q_hi, G, first, count, groups,
       status_ptr());
   return cuda_fail(cudaGetLastError(), "group_fill_kernel");
+}
+
+int launch_pool_from(const misa_problem_t& p, const uint16_t* K, float* Kbar,
+                     const int32_t* from_pos, cudaStream_t st) {
+  ProfScope ps("pool_keys", st);
+  pool_from_kernel<<<p.num_seqs, 256, 0, st>>>(K, p.key_offsets, p.block_offsets, p.block,
+                                               from_pos, Kbar, status_ptr());
+  return cuda_fail(cudaGetLastError(), "pool_from_kernel");
 }
 
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st) {
