@@ -21,6 +21,7 @@ pages publish no code).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -52,6 +53,8 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--max-queries", type=int, default=0,
                     help="keep only the last N queries (small captures for ncu)")
+    ap.add_argument("--k-cand", type=int, default=-1,
+                    help="MISA-dagger candidate count k' (default: the workload's own; 0 = off)")
     ap.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
                     help="replay each step as one CUDA graph (auto: decode workloads)")
     return ap.parse_args()
@@ -206,7 +209,7 @@ def workload_config(wl, cfg):
     c = CONFIGS[cfg]
     return {"workload": c["name"], "seqs": c["S"], "prefix_len": c["L"], "queries": wl.T,
             "H": c["H"], "d": c["d"], "pool_block": c["B"], "m": c["m"], "k": c["k"],
-            "k_cand": c["k_cand"] or None, "pairs_per_step": wl.pairs,
+            "k_cand": wl.k_cand or None, "pairs_per_step": wl.pairs,
             "l2": "inputs larger than L2 (126 MB): no flush" if wl.q_bits.nbytes + wl.K_bits.nbytes > 2 * 126e6
                   else "L2 flushed between steps (256 MB write)"}
 
@@ -291,6 +294,8 @@ def run_ours(args):
     world, rank, local = dist_init()
     cfg = args.config
     wl = make_config(cfg, seed=rank_seed(cfg, rank))
+    if args.k_cand >= 0:
+        wl = dataclasses.replace(wl, k_cand=args.k_cand)
     if args.max_queries and args.max_queries < wl.T:
         wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
     hier = bool(wl.k_cand)

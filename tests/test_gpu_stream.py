@@ -189,3 +189,27 @@ def test_stream_probe_overestimate_goes_through_fixup():
                                 Kf[:i + 1])
         ref, _ = oracle.topk(I, wl.k)
         assert set(si[i].tolist()) == set(ref.tolist()), f"row {i}"
+
+
+def test_hier_prefill_streamed_candidates_then_rerank():
+    # MISA-dagger in prefill: the coarse keep (k' = 1024) runs on the streaming
+    # scorer, then every query re-ranks its candidates with all heads.
+    wl = make_workload(seq_lens=[12000], queries="all", H=32, B=128, m=8, k=128, k_cand=1024,
+                       seed=21)
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k, k_cand=wl.k_cand)
+    misa.profile_enable(True)
+    ix.hier(q, w, K)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert "topk" in prof and "score" in prof  # streamed keep, then the rerank's top-k
+    invariants(dataclasses.replace(wl, k=wl.k_cand), ix.cand)
+    invariants(wl, ix.idx)
+    rows = sample_rows(wl, 40)
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_misa_rows(wl, rows, ix.cand[sel].cpu().numpy(), ix.cand_val[sel].cpu().numpy(),
+                           heads=ix.heads[sel].cpu().numpy(), k=wl.k_cand,
+                           m=wl.m).assert_ok()
+    parity.check_rerank_rows(wl, rows, ix.cand[sel].cpu().numpy(), ix.idx[sel].cpu().numpy(),
+                             ix.val[sel].cpu().numpy()).assert_ok()
