@@ -416,6 +416,14 @@ __device__ void final_select(uint2* region, const int* cnt, int base, int k, int
   }
 }
 
+// This CTA's j-th schedule slot.  Groups come longest first; the rounds of
+// gridDim.x slots alternate direction (CTA b takes slot b, then the round's
+// last-but-b, ...), so that every CTA's sum of group lengths is about equal.
+__device__ __forceinline__ int sched_slot(int j) {
+  const int g = (int)gridDim.x, b = (int)blockIdx.x;
+  return j * g + ((j & 1) ? g - 1 - b : b);
+}
+
 // Which group a CTA takes at schedule slot gs: longest prefix first from the
 // planner's table, or (fixup launch) one query from the failure list.
 struct Sched {
@@ -586,7 +594,7 @@ __global__ void __maxnreg__(96)
       tma_prefetch_desc(&qmap);
       int it = 0, gl = 0;
       bool ok = true;
-      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+      for (int j = 0, gs = blockIdx.x; ok && gs < count; gs = sched_slot(++j)) {
         const int4 grp = fetch_group(sc, count, gs);
         if (grp.w < 0) continue;  // no valid query in the group
         const int64_t key_base = ko[grp.x];
@@ -622,7 +630,7 @@ __global__ void __maxnreg__(96)
       const uint32_t q_addr = smem_u32(s.q);
       int it = 0, tb = 0, gl = 0;
       bool ok = true;
-      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+      for (int j = 0, gs = blockIdx.x; ok && gs < count; gs = sched_slot(++j)) {
         const int4 grp = fetch_group(sc, count, gs);
         if (grp.w < 0) continue;
         const int ntiles = (grp.w + kTileKeys) / kTileKeys;
@@ -664,7 +672,7 @@ __global__ void __maxnreg__(96)
     uint32_t ephase = 0;
     int tb = 0;
     bool ok = true;
-    for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+    for (int j = 0, gs = blockIdx.x; ok && gs < count; gs = sched_slot(++j)) {
       const int4 grp = fetch_group(sc, count, gs);
       if (grp.w < 0) continue;
       const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
@@ -856,7 +864,7 @@ __global__ void __maxnreg__(96)
     uint32_t* selh = s.sel + sw * kSelBins;
     int gl = 0;
     bool ok = true;
-    for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+    for (int j = 0, gs = blockIdx.x; ok && gs < count; gs = sched_slot(++j)) {
       const int4 grp = fetch_group(sc, count, gs);
       if (grp.w < 0) continue;
       const int nq = grp.z - grp.y;
