@@ -11,7 +11,8 @@
 // score leaves the SM unless it can still be in its query's top-k.
 //
 // CTA (persistent, one per SM): query groups of G = 256/m queries taken
-// longest-prefix first, round-robin over CTAs.  Per group: the group's
+// longest-prefix first, in rounds over the CTAs that alternate direction.
+// Per group: the group's
 // (query, head) rows stay in shared memory (B operand, N = 256); 128-key
 // tiles of K stream through a 4-stage TMA ring (A operand); tcgen05.mma
 // accumulates 128 keys x 256 columns in TMEM, two buffers.
@@ -19,9 +20,10 @@
 // Epilogue (16 warps, four per SM sub-partition so that their dependency
 // chains overlap: TMEM lane quarter = warp % 4, column quarter = which of the
 // four warps of that lane quarter, i.e. 64 columns = 64/m queries each), per
-// tile: tcgen05.ld of 32 columns, wait, then per key and query
-// I = sum_j w_j ReLU(acc_j) (the TMEM buffer is released after the warp's
-// last load), the causal mask, and the streaming selection:
+// tile: four 16-column tcgen05.ld, each issued before the previous chunk is
+// summed, then per key and query I = sum_j w_j ReLU(acc_j) (the TMEM buffer
+// is released after the warp's last load), the causal mask, and the
+// streaming selection:
 //   * probe: a group first scores every 24th tile of its prefix and keeps a
 //     256-bin histogram per query (1/32-octave bins of the order-preserving
 //     score key, from 7 octaves below the first scored tile's maximum to one
@@ -32,11 +34,12 @@
 //     of the prefix), i.e. a few standard deviations below the expected k-th
 //     best score.
 //   * main pass over all tiles: a key is appended to query q's candidates
-//     only if I >= tau_q.  Each (query, TMEM lane) has its own list with one
-//     row per tile, so nothing can overflow and no lane needs a rank from
-//     the others: a passing lane stores to row cnt of its list and counts
-//     (a predicated store and an add, no vote).  A query's 128 lists are
-//     stored row by row, so that a row of all lists is 1 KB contiguous.
+//     only if I >= tau_q.  Each (query, TMEM lane) has its own list, so no
+//     lane needs a rank from the others: a passing lane stores to row cnt of
+//     its list and counts (a predicated store and an add, no vote).  Lists
+//     hold kRowsCap rows; a fuller list stops storing and sends its query to
+//     the rescan.  A query's 128 lists are stored row by row, so that a row
+//     of all lists is 1 KB contiguous.
 //   * check and select, by two selector warps while the epilogue warps
 //     already stream the next group (the candidate lists are double
 //     buffered; when the selectors fall behind, the epilogue warps claim the
