@@ -20,7 +20,9 @@
 // released as soon as it is copied to registers.  The causal partial block
 // of every key position (the running mean of its block up to that key) is
 // computed beforehand by one warp per pooled block, so each query only
-// reads its row.
+// reads its row.  Persistent: one CTA per SM walks its groups; the next
+// group's q rows load as soon as the current group's MMAs are done, and its
+// MMAs start while the epilogue still ranks the current group's heads.
 #include "common.cuh"
 #include "internal.h"
 
@@ -50,6 +52,7 @@ struct Smem {
   uint64_t* tfull;
   uint64_t* tempty;  // [4]
   uint64_t* qfull;
+  uint64_t* qempty;
   uint64_t* drain;
   uint32_t* tmem_slot;
   int* abort;
@@ -70,7 +73,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tfull = bars + 2 * kStages;
   s.tempty = s.tfull + 1;
   s.qfull = s.tempty + 4;
-  s.drain = s.qfull + 1;
+  s.qempty = s.qfull + 1;
+  s.drain = s.qempty + 1;
   s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
   return s;
@@ -138,26 +142,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int G = (kRows / H) < kMaxG ? (kRows / H) : kMaxG;
   constexpr int ROWS = G * H;                       // rows used (<= 512)
   constexpr int NSUB = (ROWS + 127) / 128;          // accumulators used
+  constexpr uint32_t kQTx = 2u * ((ROWS + 31) / 32) * 32u * 128u;
   extern __shared__ uint8_t smem_raw[];
 
-  const int gi = blockIdx.x;
-  if (gi >= *group_count) return;
-  const int4 grp = groups[gi];
-  const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
-  if (grp.w < 0 || nq <= 0) {
-    // no valid query: deterministic padding for every row of the group
-    for (int i = threadIdx.x; i < nq * m; i += blockDim.x) {
-      heads[(int64_t)qb * m + i] = -1;
-      w_r[(int64_t)qb * m + i] = 0.f;
-    }
-    for (int i = threadIdx.x; i < nq * m * (kD / 8); i += blockDim.x)
-      reinterpret_cast<uint4*>(q_r + (int64_t)qb * m * kD)[i] = make_uint4(0, 0, 0, 0);
-    return;
-  }
-  const int64_t L = ko[seq + 1] - ko[seq];
-  const int64_t blk0 = bo[seq];
-  const int max_full = (grp.w + 1) / B;
-  const int nchunks = (max_full + kChunk - 1) / kChunk;
+  // Persistent: CTA b takes groups b, b + gridDim.x, ...; every role walks
+  // the same sequence and skips the same groups (no valid query).
+  const int count = *group_count;
+  if ((int)blockIdx.x >= count) return;
 
   Smem s = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -170,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(s.tfull, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&s.tempty[i], 4);
     mbar_init(s.qfull, 1);
+    mbar_init(s.qempty, 1);
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
@@ -177,15 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(s.tmem_slot, 512);
     tmem_relinquish();
-  }
-  if (warp >= 2 && threadIdx.x - 64 < kMaxG) {
-    const int qi = threadIdx.x - 64;
-    int p = -1;
-    if (qi < nq) {
-      p = q_pos[qb + qi];
-      if (p < 0 || p >= L) p = -1;
-    }
-    s.pos[qi] = p;
   }
   tc_fence_before();
   __syncthreads();
@@ -196,64 +179,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
-      mbar_arrive_expect_tx(s.qfull, 2u * ((ROWS + 31) / 32) * 32u * 128u);
-      for (int h = 0; h < 2; ++h)
-        for (int r0 = 0; r0 < ROWS; r0 += 32)
-          tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64, qb * H + r0);
-      int it = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        for (int part = 0; part < 2; ++part, ++it) {
-          const int st = it % kStages;
-          if (!mbar_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, s.abort, status)) {
-            c = nchunks;
-            break;
+      tma_prefetch_desc(&himap);
+      tma_prefetch_desc(&lomap);
+      int it = 0, gl = 0;
+      bool ok = true;
+      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+        const int4 grp = groups[gs];
+        if (grp.w < 0 || grp.z <= grp.y) continue;
+        const int64_t blk0 = bo[grp.x];
+        const int nchunks = ((grp.w + 1) / B + kChunk - 1) / kChunk;
+        // The q rows are replaced once the previous group's MMAs are done.
+        if (!(ok = mbar_wait(s.qempty, (gl & 1) ^ 1, s.abort, status))) break;
+        mbar_arrive_expect_tx(s.qfull, kQTx);
+        for (int h = 0; h < 2; ++h)
+          for (int r0 = 0; r0 < ROWS; r0 += 32)
+            tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
+                        grp.y * H + r0);
+        ++gl;
+        for (int c = 0; ok && c < nchunks; ++c) {
+          for (int part = 0; part < 2; ++part, ++it) {
+            const int st = it % kStages;
+            if (!(ok = mbar_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, s.abort, status))) break;
+            mbar_arrive_expect_tx(&s.full[st], kStageBytes);
+            const CUtensorMap* mp = part == 0 ? &himap : &lomap;
+            const int32_t row = (int32_t)(blk0 + (int64_t)c * kChunk);
+            uint8_t* dst = s.k + st * kStageBytes;
+            tma_load_2d(mp, &s.full[st], dst, 0, row);
+            tma_load_2d(mp, &s.full[st], dst + kHalfBytes, 64, row);
           }
-          mbar_arrive_expect_tx(&s.full[st], kStageBytes);
-          const CUtensorMap* mp = part == 0 ? &himap : &lomap;
-          const int32_t row = (int32_t)(blk0 + (int64_t)c * kChunk);
-          uint8_t* dst = s.k + st * kStageBytes;
-          tma_load_2d(mp, &s.full[st], dst, 0, row);
-          tma_load_2d(mp, &s.full[st], dst + kHalfBytes, 64, row);
         }
       }
       for (int i = max(0, it - kStages); i < it; ++i)
         mbar_wait(&s.full[i % kStages], (i / kStages) & 1, s.abort, status, kDrainCycles, true);
-      mbar_wait(s.qfull, 0, s.abort, status, kDrainCycles, true);
+      if (gl > 0) mbar_wait(s.qfull, (gl - 1) & 1, s.abort, status, kDrainCycles, true);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, kChunk);
       const uint32_t q_addr = smem_u32(s.q);
-      bool ok = mbar_wait(s.qfull, 0, s.abort, status);
-      tc_fence_after();
-      int it = 0;
-      for (int c = 0; ok && c < nchunks; ++c) {
-        for (int part = 0; ok && part < 2; ++part, ++it) {
-          const int st = it % kStages;
-          if (!(ok = mbar_wait(&s.full[st], (it / kStages) & 1, s.abort, status))) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(s.k + st * kStageBytes);
+      int it = 0, cc = 0, gl = 0;
+      bool ok = true;
+      for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+        const int4 grp = groups[gs];
+        if (grp.w < 0 || grp.z <= grp.y) continue;
+        const int nchunks = ((grp.w + 1) / B + kChunk - 1) / kChunk;
+        if (!(ok = mbar_wait(s.qfull, gl & 1, s.abort, status))) break;
+        tc_fence_after();
+        for (int c = 0; ok && c < nchunks; ++c, ++cc) {
+          for (int part = 0; ok && part < 2; ++part, ++it) {
+            const int st = it % kStages;
+            if (!(ok = mbar_wait(&s.full[st], (it / kStages) & 1, s.abort, status))) break;
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(s.k + st * kStageBytes);
 #pragma unroll
-          for (int sub = 0; sub < NSUB; ++sub) {
-            if (part == 0 &&
-                !(ok = mbar_wait(&s.tempty[sub], (c & 1) ^ 1, s.abort, status)))
-              break;
-            if (part == 0) tc_fence_after();
-            const uint32_t d = tmem_base + sub * kChunk;
+            for (int sub = 0; sub < NSUB; ++sub) {
+              // accumulator `sub` is free once the epilogue has read chunk cc-1
+              if (part == 0 &&
+                  !(ok = mbar_wait(&s.tempty[sub], (cc & 1) ^ 1, s.abort, status)))
+                break;
+              if (part == 0) tc_fence_after();
+              const uint32_t d = tmem_base + sub * kChunk;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk & 3) * 32;
-              const uint64_t a = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes +
-                                                   sub * 128 * 128 + off);
-              const uint64_t b = sw128_kmajor_desc(k_addr + (kk >> 2) * kHalfBytes + off);
-              umma_bf16(d, a, b, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t a = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes +
+                                                     sub * 128 * 128 + off);
+                const uint64_t b = sw128_kmajor_desc(k_addr + (kk >> 2) * kHalfBytes + off);
+                umma_bf16(d, a, b, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+              }
             }
+            if (!ok) break;
+            umma_commit(&s.empty[st]);
           }
-          if (!ok) break;
-          umma_commit(&s.empty[st]);
+          if (ok) umma_commit(s.tfull);
         }
-        if (ok) umma_commit(s.tfull);
+        umma_commit(s.qempty);  // q rows free once this group's MMAs are done
+        ++gl;
       }
       umma_commit(s.drain);
       mbar_wait(s.drain, 0, s.abort, status, kDrainCycles, true);
@@ -263,60 +265,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;            // 0..127
     const int quarter = warp & 3;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-
-    // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
-    // of every accumulator.
-    float acc[NSUB];
-    int lim[NSUB];
-#pragma unroll
-    for (int sub = 0; sub < NSUB; ++sub) {
-      acc[sub] = 0.f;
-      const int row = sub * 128 + quarter * 32 + lane;
-      const int qi = row / H;
-      const int p = (row < ROWS && qi < nq) ? s.pos[qi] : -1;
-      lim[sub] = (p + 1) / B;  // number of full blocks visible to this row
-    }
+    int cc = 0;
     bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      if (!(ok = warp_wait(s.tfull, c & 1, s.abort, status))) break;
-      tc_fence_after();
+    for (int gs = blockIdx.x; ok && gs < count; gs += gridDim.x) {
+      const int4 grp = groups[gs];
+      const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
+      if (grp.w < 0 || nq <= 0) {
+        // no valid query: deterministic padding for every row of the group
+        for (int i = et; i < nq * m; i += 128) {
+          heads[(int64_t)qb * m + i] = -1;
+          w_r[(int64_t)qb * m + i] = 0.f;
+        }
+        for (int i = et; i < nq * m * (kD / 8); i += 128)
+          reinterpret_cast<uint4*>(q_r + (int64_t)qb * m * kD)[i] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      const int64_t L = ko[seq + 1] - ko[seq];
+      const int nchunks = ((grp.w + 1) / B + kChunk - 1) / kChunk;
+      if (et < kMaxG) {
+        int p = -1;
+        if (et < nq) {
+          p = q_pos[qb + et];
+          if (p < 0 || p >= L) p = -1;
+        }
+        s.pos[et] = p;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+
+      // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
+      // of every accumulator.
+      float acc[NSUB];
+      int lim[NSUB];
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
-        float v[4][32];
+        acc[sub] = 0.f;
+        const int row = sub * 128 + quarter * 32 + lane;
+        const int qi = row / H;
+        const int p = (row < ROWS && qi < nq) ? s.pos[qi] : -1;
+        lim[sub] = (p + 1) / B;  // number of full blocks visible to this row
+      }
+      for (int c = 0; c < nchunks && ok; ++c, ++cc) {
+        if (!(ok = warp_wait(s.tfull, cc & 1, s.abort, status))) break;
+        tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld32(lane_addr + sub * kChunk + j * 32, v[j]);
-        tmem_wait_ld();
+        for (int sub = 0; sub < NSUB; ++sub) {
+          float v[4][32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) reg_fence32(v[j]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.tempty[sub]);
-        const int nvis = lim[sub] - c * kChunk;  // visible columns of this chunk
-        if (nvis >= kChunk) {
-          float a0 = 0.f, a1 = 0.f;
+          for (int j = 0; j < 4; ++j) tmem_ld32(lane_addr + sub * kChunk + j * 32, v[j]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 4; ++j) reg_fence32(v[j]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[sub]);
+          const int nvis = lim[sub] - c * kChunk;  // visible columns of this chunk
+          if (nvis >= kChunk) {
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              a0 += fmaxf(v[j][x], 0.f);
-              a1 += fmaxf(v[j][x + 1], 0.f);
-            }
-          acc[sub] += a0 + a1;
-        } else if (nvis > 0) {
-          float a0 = 0.f;
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+              for (int x = 0; x < 32; x += 2) {
+                a0 += fmaxf(v[j][x], 0.f);
+                a1 += fmaxf(v[j][x + 1], 0.f);
+              }
+            acc[sub] += a0 + a1;
+          } else if (nvis > 0) {
+            float a0 = 0.f;
 #pragma unroll
-            for (int x = 0; x < 32; ++x)
-              if (j * 32 + x < nvis) a0 += fmaxf(v[j][x], 0.f);
-          acc[sub] += a0;
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int x = 0; x < 32; ++x)
+                if (j * 32 + x < nvis) a0 += fmaxf(v[j][x], 0.f);
+            acc[sub] += a0;
+          }
         }
       }
-    }
+      if (!ok) break;
 
-    // Epilogue threads sync on named barrier 1 (only these 128 threads).
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok) {
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
         const int row = sub * 128 + quarter * 32 + lane;
@@ -353,9 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         s.r[row] = r;
       }
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       // Top-m per query by (r desc, head asc): rank of each head.
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
@@ -390,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kD / 8; ++i) dst[i] = __ldg(src + i);
         }
       }
+      // s.pos and s.r are rewritten by the next group
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   }
 
@@ -409,7 +434,8 @@ int launch_h(const RouteTcArgs& a, const CUtensorMap& qmap, const CUtensorMap& h
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
   ProfScope ps("route", st);
-  kern<<<a.max_groups, kThreads, kSmemBytes, st>>>(
+  const int grid = a.max_groups < num_sms() ? a.max_groups : num_sms();  // persistent
+  kern<<<grid, kThreads, kSmemBytes, st>>>(
       qmap, himap, lomap, a.q, a.w, a.K, a.p->key_offsets, a.p->block_offsets, a.p->q_pos,
       a.groups, a.group_count, a.Pm, a.p->block, a.m, a.heads, a.q_r, a.w_r, a.router_scores,
       status_ptr());
