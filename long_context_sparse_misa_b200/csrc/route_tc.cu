@@ -39,12 +39,13 @@ constexpr int kQHalfBytes = kRows * 128;              // 64 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kMaxG = 16;                             // queries per group
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kRows * 4 /*r*/ +
-                           kMaxG * 4 * 2 + 16 * 8 + 16;
+                           kMaxG * kD * 4 /*pm*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
 
 struct Smem {
   uint8_t* q;
   uint8_t* k;
   float* r;   // [kRows] router scores of the group
+  float* pm;  // [kMaxG][128] running block means at the group's query positions
   int* pos;
   int* flags;
   uint64_t* full;
@@ -65,7 +66,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.q = p;
   s.k = p + kQBytes;
   s.r = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
-  s.pos = reinterpret_cast<int*>(s.r + kRows);
+  s.pm = s.r + kRows;
+  s.pos = reinterpret_cast<int*>(s.pm + kMaxG * kD);
   s.flags = s.pos + kMaxG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
   s.full = bars;
@@ -291,6 +293,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         s.pos[et] = p;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
+      // The queries' running block means (partial block), staged for the
+      // head rows of each query (coalesced 16-byte loads).
+      for (int i = et; i < nq * (kD / 4); i += 128) {
+        const int qi = i / (kD / 4), c4 = i - qi * (kD / 4);
+        const int p = s.pos[qi];
+        if (p >= 0 && (p + 1) % B != 0)
+          reinterpret_cast<float4*>(s.pm + qi * kD)[c4] =
+              __ldg(reinterpret_cast<const float4*>(Pm + (ko[seq] + p) * kD) + c4);
+      }
 
       // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
       // of every accumulator.
@@ -341,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // s.pm complete
 
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
@@ -353,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float total = acc[sub];
           if ((p + 1) % B != 0) {
             const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)(qb + qi) * H + h) * kD);
-            const float* Pq = Pm + (ko[seq] + p) * kD;  // running block mean at p
+            const float* Pq = s.pm + qi * kD;  // running block mean at p
             float dp = 0.f;
 #pragma unroll
             for (int i = 0; i < kD / 8; ++i) {
