@@ -83,3 +83,10 @@ def test_host_argument_errors_without_gpu(misa):
     assert lib.misa_route(rp, 16, 16, 16, 16, 8, 16, 16, 16, None, 16, 8, None) == 3
     assert lib.misa_selftest_timeout(0, None) == 1
     assert lib.misa_block_offsets(None, 1, 64, None, None) == 1
+    # incremental pooling: NULL / misaligned arguments are rejected on the host
+    assert lib.misa_pool_keys_from(rp, 16, 16, None, None) == 1
+    assert b"from_pos" in lib.misa_last_error_string()
+    assert lib.misa_pool_keys_from(rp, 16, 16, 18, None) == 1
+    assert lib.misa_pool_keys_from(rp, 16, None, 16, None) == 1
+    # the static-scratch router validates like misa_route and refuses m > H
+    assert lib.misa_route_static(rp, 16, 16, 16, 16, 65, 16, 16, 16, None, None) == 1
