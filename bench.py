@@ -71,9 +71,11 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-def score_src_sha():
+def score_src_sha(kernel: str = "score_stream"):
+    """Hash of the sources that one scoring kernel is compiled from."""
+    main = "score_stream.cu" if kernel == "score_stream" else "score.cu"
     h = hashlib.sha256()
-    for f in ("score.cu", "score_stream.cu", "common.cuh", "internal.h"):
+    for f in (main, "common.cuh", "internal.h"):
         with open(os.path.join(ROOT, "long_context_sparse_misa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -85,7 +87,7 @@ def traffic_per_pair(kernel: str, workload: str):
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
-    sha = score_src_sha()
+    sha = score_src_sha(kernel)
     for fn in sorted(os.listdir(pdir)):
         if not fn.endswith(".md"):
             continue
@@ -102,23 +104,30 @@ def traffic_per_pair(kernel: str, workload: str):
 
 
 class Clocks:
-    """Samples nvidia-smi every 100 ms while the timed region runs."""
+    """Samples nvidia-smi every 20 ms; the summary covers the samples taken
+    between begin() and end() (the timed region)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, uuid):
         self.uuid, self.proc, self.lines = uuid, None, []
+        self.i0 = self.i1 = 0
 
     def start(self):
+        """Starts the sampler and waits (up to 10 s) for its first sample."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 10 and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
 
@@ -126,9 +135,23 @@ class Clocks:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def begin(self):
+        self.i0 = len(self.lines)
+
+    def end(self):
+        self.i1 = len(self.lines)
+
     def stop(self):
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        note = None
+        if self.i1 <= self.i0:
+            # Region shorter than the sampling period: take the next sample.
+            t0 = time.time()
+            while len(self.lines) <= self.i1 and time.time() - t0 < 1.0:
+                time.sleep(0.005)
+            self.i1 = min(len(self.lines), self.i0 + 1)
+            note = "timed region shorter than the sampling period: first sample after it"
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -137,7 +160,7 @@ class Clocks:
         self.t.join(timeout=2)
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[self.i0:self.i1]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -149,8 +172,11 @@ class Clocks:
             for n, v in zip(names, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+               "samples": len(sm), "period_ms": self.PERIOD_MS, "reasons": sorted(reasons)}
+        if note:
+            out["note"] = note
+        return out
 
 
 def dist_init(backend: str = "nccl"):
@@ -211,7 +237,9 @@ def workload_config(wl, cfg):
             "H": c["H"], "d": c["d"], "pool_block": c["B"], "m": c["m"], "k": c["k"],
             "k_cand": wl.k_cand or None, "pairs_per_step": wl.pairs,
             "l2": "inputs larger than L2 (126 MB): no flush" if wl.q_bits.nbytes + wl.K_bits.nbytes > 2 * 126e6
-                  else "L2 flushed between steps (256 MB write)"}
+                  else "L2 flushed between steps (256 MB write, then a 256 MB read of another buffer)",
+            "launch": "a ~1 ms device sleep before each timed step keeps the stream busy, "
+                      "so the events bracket device time and not host launch latency"}
 
 
 # ------------------------------------------------------------------ CPU oracle sample
@@ -320,11 +348,26 @@ def run_ours(args):
     eager_run = run
     small_inputs = wl.q_bits.nbytes + wl.K_bits.nbytes < 2 * 126e6
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small_inputs else None
+    # Read after the write: the flush's own dirty lines are written back here,
+    # outside the timed step, and L2 is left holding clean unrelated lines.
+    clean = torch.ones(64 << 20, dtype=torch.int32, device=dev) if small_inputs else None
 
-    def step():
+    def l2_flush():
         if flush is not None:
             flush.fill_(1)
+            clean.sum()
+
+    def step():
+        l2_flush()
         run()
+
+    def settle():
+        """Between timed intervals: the L2 flush (small inputs only), then a
+        ~1 ms device sleep so that the host has queued the whole next step
+        before the device reaches it; the events then bracket device time,
+        not the host's launch latency."""
+        l2_flush()
+        torch.cuda._sleep(2_000_000)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -354,19 +397,20 @@ def run_ours(args):
     clocks = Clocks(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
     torch.cuda.synchronize()
     barrier(world)
-    misa.profile_enable(graph is None)
     clocks.start()
+    misa.profile_enable(graph is None)
+    clocks.begin()
     # Each step is bracketed by its own events; the L2 flush (small inputs
     # only) runs between steps, outside the timed intervals.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for e0, e1 in evs:
-        if flush is not None:
-            flush.fill_(1)
+        settle()
         e0.record()
         run()
         e1.record()
     torch.cuda.synchronize()
+    clocks.end()
     clk = clocks.stop()
     prof = misa.profile_collect()
     misa.profile_enable(False)
@@ -381,8 +425,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         misa.profile_enable(True)
         for _ in range(args.steps):
-            if flush is not None:
-                flush.fill_(1)
+            settle()
             eager_run()
         torch.cuda.synchronize()
         prof = misa.profile_collect()
@@ -452,8 +495,7 @@ def run_ours(args):
     if not args.no_dense:
         dense_steps = max(1, min(args.steps, 5))
         for _ in range(1):
-            if flush is not None:
-                flush.fill_(1)
+            l2_flush()
             ix.dense(q, w, K)
         torch.cuda.synchronize()
         dense_run = lambda: ix.dense(q, w, K)
@@ -465,8 +507,7 @@ def run_ours(args):
         devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(dense_steps)]
         for e0, e1 in devs:
-            if flush is not None:
-                flush.fill_(1)
+            settle()
             e0.record()
             dense_run()
             e1.record()
@@ -477,6 +518,7 @@ def run_ours(args):
         if dgraph is not None:
             misa.profile_enable(True)
             for _ in range(dense_steps):
+                settle()
                 ix.dense(q, w, K)
             torch.cuda.synchronize()
             dprof = misa.profile_collect()

@@ -106,6 +106,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* a
   }
 }
 
+// ---------------------------------------------------------------- dependent launch
+// First statement of a kernel that may be launched with programmatic
+// dependent launch: wait until the previous kernel on the stream has
+// completed and its writes are visible (returns at once when launched
+// normally), then let the next kernel's CTAs be scheduled.  The next kernel
+// waits in turn, so no kernel runs ahead of one that it may depend on.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

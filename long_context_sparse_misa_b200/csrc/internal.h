@@ -29,6 +29,26 @@ uint32_t* status_ptr();
 int make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 int set_smem_limit(const void* kernel, int bytes);
+
+// Launches `kern` with programmatic dependent launch: its CTAs may be
+// scheduled while the previous kernel on `st` is still finishing.  Every
+// kernel launched this way calls pdl_wait() (common.cuh) before it reads or
+// writes global memory, so the result is the same as with plain stream order.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 // SMs of the current device.
 int num_sms();
 // Workspace misa_route uses on its fastest path for a checked problem.

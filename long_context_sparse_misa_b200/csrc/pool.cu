@@ -62,6 +62,7 @@ __global__ void block_offsets_kernel(const int64_t* __restrict__ ko, int S, int 
 // max_pos.
 __global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_lo, int q_hi,
                                   int G, int* __restrict__ first, int* __restrict__ count) {
+  pdl_wait_then_release();
   __shared__ int warp_sums[32];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
@@ -107,6 +108,7 @@ __global__ void group_fill_kernel(const int64_t* __restrict__ ko, const int32_t*
                                   int G, const int* __restrict__ first,
                                   const int* __restrict__ count, int4* __restrict__ groups,
                                   uint32_t* status) {
+  pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int fg = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
   if (fg >= *count) return;
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(256) pool_from_kernel(const uint16_t* __restri
                                                         const int32_t* __restrict__ from_pos,
                                                         float* __restrict__ Kbar,
                                                         uint32_t* status) {
+  pdl_wait_then_release();
   const int s = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int64_t L = ko[s + 1] - ko[s];
@@ -244,23 +247,24 @@ int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4*
                        int* count, cudaStream_t st) {
   ProfScope ps("plan_groups", st);
   int* first = count + 4;  // [S] after the count word (see groups_bytes)
-  group_scan_kernel<<<1, 1024, 0, st>>>(p.query_offsets, p.num_seqs, q_lo, q_hi, G, first, count);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(group_scan_kernel, dim3(1), dim3(1024), 0, st, p.query_offsets,
+                             p.num_seqs, q_lo, q_hi, G, first, count);
   if (e != cudaSuccess) return cuda_fail(e, "group_scan_kernel");
   const int64_t max_groups = (int64_t)(q_hi - q_lo + G - 1) / G + p.num_seqs;
   const int warps = 8;
-  group_fill_kernel<<<(unsigned)((max_groups + warps - 1) / warps), warps * 32, 0, st>>>(
-      p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo, q_hi, G, first, count, groups,
-      status_ptr());
-  return cuda_fail(cudaGetLastError(), "group_fill_kernel");
+  e = launch_pdl(group_fill_kernel, dim3((unsigned)((max_groups + warps - 1) / warps)),
+                 dim3(warps * 32), 0, st, p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs,
+                 q_lo, q_hi, G, (const int*)first, (const int*)count, groups, status_ptr());
+  return cuda_fail(e, "group_fill_kernel");
 }
 
 int launch_pool_from(const misa_problem_t& p, const uint16_t* K, float* Kbar,
                      const int32_t* from_pos, cudaStream_t st) {
   ProfScope ps("pool_keys", st);
-  pool_from_kernel<<<p.num_seqs, 256, 0, st>>>(K, p.key_offsets, p.block_offsets, p.block,
-                                               from_pos, Kbar, status_ptr());
-  return cuda_fail(cudaGetLastError(), "pool_from_kernel");
+  return cuda_fail(launch_pdl(pool_from_kernel, dim3(p.num_seqs), dim3(256), 0, st, K,
+                              p.key_offsets, p.block_offsets, p.block, from_pos, Kbar,
+                              status_ptr()),
+                   "pool_from_kernel");
 }
 
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st) {

@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
                  int32_t* __restrict__ heads, uint16_t* __restrict__ q_r, float* __restrict__ w_r,
                  float* __restrict__ router_scores, uint32_t* status, int nsplit_max,
                  int sms, float* __restrict__ partial) {
+  pdl_wait_then_release();
   extern __shared__ __align__(16) float smem_f[];
   float* kb = smem_f;                         // [kChunk][128]
   float* part = kb + kChunk * kD;             // [G][128]
@@ -119,15 +120,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
         for (int i = 0; i < kD / 4; i += 2) {
+          // packed pairs: d0 takes dims 0 mod 4 and 2 mod 4 in order, d1
+          // dims 1 and 3 mod 4, d2 / d3 the same on the next four
           const float4 a = row[i], c = row[i + 1];
-          d0 = fmaf(qreg[4 * i + 0], a.x, d0);
-          d1 = fmaf(qreg[4 * i + 1], a.y, d1);
-          d0 = fmaf(qreg[4 * i + 2], a.z, d0);
-          d1 = fmaf(qreg[4 * i + 3], a.w, d1);
-          d2 = fmaf(qreg[4 * i + 4], c.x, d2);
-          d3 = fmaf(qreg[4 * i + 5], c.y, d3);
-          d2 = fmaf(qreg[4 * i + 6], c.z, d2);
-          d3 = fmaf(qreg[4 * i + 7], c.w, d3);
+          ffma2(d0, d1, qreg[4 * i + 0], qreg[4 * i + 1], a.x, a.y);
+          ffma2(d0, d1, qreg[4 * i + 2], qreg[4 * i + 3], a.z, a.w);
+          ffma2(d2, d3, qreg[4 * i + 4], qreg[4 * i + 5], c.x, c.y);
+          ffma2(d2, d3, qreg[4 * i + 6], qreg[4 * i + 7], c.z, c.w);
         }
         acc += fmaxf((d0 + d1) + (d2 + d3), 0.f);
       }
@@ -262,11 +261,12 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
   if (nsplit <= 1 || !partial) {
     if ((rc = set_smem_limit((const void*)route_kernel<kWhole>, smem))) return rc;
     ProfScope ps("route", st);
-    route_kernel<kWhole><<<max_groups, kRouteThreads, smem, st>>>(
-        q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
-        p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), 1, sms,
-        nullptr);
-    return cuda_fail(cudaGetLastError(), "route_kernel");
+    return cuda_fail(launch_pdl(route_kernel<kWhole>, dim3(max_groups), dim3(kRouteThreads),
+                                smem, st, q, w, K, Kbar, p.key_offsets, p.block_offsets,
+                                p.q_pos, groups, group_count, p.num_heads, p.block, m, G, heads,
+                                q_r, w_r, router_scores, status_ptr(), 1, sms,
+                                (float*)nullptr),
+                     "route_kernel");
   }
   if ((rc = set_smem_limit((const void*)route_kernel<kPartial>, smem))) return rc;
   if ((rc = set_smem_limit((const void*)route_kernel<kFinish>, smem))) return rc;
@@ -274,18 +274,20 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
     // One CTA per (group, range) and one per group for its partial block;
     // the device uses the first count * (ns + 1) of them.
     ProfScope ps("route", st);
-    route_kernel<kPartial><<<max_groups * (nsplit + 1), kRouteThreads, smem, st>>>(
-        q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
-        p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), nsplit, sms,
-        partial);
-    if ((rc = cuda_fail(cudaGetLastError(), "route_kernel (ranges)"))) return rc;
+    rc = cuda_fail(launch_pdl(route_kernel<kPartial>, dim3(max_groups * (nsplit + 1)),
+                              dim3(kRouteThreads), smem, st, q, w, K, Kbar, p.key_offsets,
+                              p.block_offsets, p.q_pos, groups, group_count, p.num_heads,
+                              p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(),
+                              nsplit, sms, partial),
+                   "route_kernel (ranges)");
+    if (rc) return rc;
   }
   ProfScope ps("route_finish", st);
-  route_kernel<kFinish><<<max_groups, kRouteThreads, smem, st>>>(
-      q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups, group_count,
-      p.num_heads, p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(), nsplit, sms,
-      partial);
-  return cuda_fail(cudaGetLastError(), "route_kernel (finish)");
+  return cuda_fail(launch_pdl(route_kernel<kFinish>, dim3(max_groups), dim3(kRouteThreads),
+                              smem, st, q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos,
+                              groups, group_count, p.num_heads, p.block, m, G, heads, q_r, w_r,
+                              router_scores, status_ptr(), nsplit, sms, partial),
+                   "route_kernel (finish)");
 }
 
 }  // namespace misa

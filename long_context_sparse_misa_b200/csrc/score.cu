@@ -82,21 +82,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                  const int32_t* __restrict__ cand, int k_cand, const int4* __restrict__ groups,
                  const int* __restrict__ group_count, int tiles_per_split, int q_lo,
                  float* __restrict__ I, int64_t ld, int64_t total_keys, uint32_t* status) {
+  pdl_wait_then_release();
   constexpr int G = GATHER ? 1 : kMaxN / MH;
   static_assert(G * MH <= kMaxN, "group too wide");
   extern __shared__ uint8_t smem_raw[];
 
-  const int gi = blockIdx.x;
-  if (gi >= *group_count) return;
+  // tiles_per_split > 0: CTA (x, y) takes group x, tiles from y * tiles_per_split.
+  // tiles_per_split == 0: one wave of gridDim.x CTAs spread over the groups
+  // that exist, gridDim.x / count consecutive CTAs per group.
+  const int count = *group_count;
+  int gi = blockIdx.x, split = blockIdx.y, nsplit = 0;
+  if (tiles_per_split == 0) {
+    nsplit = count > 0 ? max(1, (int)gridDim.x / count) : 1;
+    gi = blockIdx.x / nsplit;
+    split = blockIdx.x % nsplit;
+  }
+  if (gi >= count) return;
   const int4 grp = groups[gi];
   const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y, maxpos = grp.w;
   if (maxpos < 0 || nq <= 0) return;
   const int64_t key_base = ko[seq];
   const int ntiles = GATHER ? (k_cand + kTileKeys - 1) / kTileKeys
                             : (maxpos + 1 + kTileKeys - 1) / kTileKeys;
-  const int tile0 = blockIdx.y * tiles_per_split;
+  const int tps = tiles_per_split > 0 ? tiles_per_split : (ntiles + nsplit - 1) / nsplit;
+  const int tile0 = split * tps;
   if (tile0 >= ntiles) return;
-  const int nt = min(ntiles, tile0 + tiles_per_split) - tile0;
+  const int nt = min(ntiles, tile0 + tps) - tile0;
   const int NP = ((nq * MH + 31) / 32) * 32;  // MMA N (multiple of 32, <= 256)
 
   Smem s = carve(smem_raw);
@@ -115,6 +126,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
+  }
+  // Contiguous mode: the producer thread starts the query rows and the first
+  // kStages key tiles at once (the stages start empty), before the block-wide
+  // set-up below, so the first loads overlap it.
+  int pre = 0;
+  if (!GATHER && threadIdx.x == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
+    mbar_arrive_expect_tx(s.qfull, 2u * NP * 128u);
+    for (int h = 0; h < 2; ++h)
+      for (int r0 = 0; r0 < NP; r0 += 32)
+        tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64, qb * MH + r0);
+    pre = min(kStages, nt);
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&s.full[i], kStageBytes);
+      const int32_t krow = (int32_t)(key_base + (int64_t)(tile0 + i) * kTileKeys);
+      uint8_t* dst = s.k + i * kStageBytes;
+      tma_load_2d(&kmap, &s.full[i], dst, 0, krow);
+      tma_load_2d(&kmap, &s.full[i], dst + kHalfBytes, 64, krow);
+    }
   }
   if (warp == 1) {
     tmem_alloc(s.tmem_slot, kTmemCols);
@@ -146,15 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (!GATHER) {
       if (lane == 0) {
-        tma_prefetch_desc(&kmap);
-        tma_prefetch_desc(&qmap);
-        mbar_arrive_expect_tx(s.qfull, 2u * NP * 128u);
-        for (int h = 0; h < 2; ++h)
-          for (int r0 = 0; r0 < NP; r0 += 32)
-            tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
-                        qb * MH + r0);
-        int issued = 0;
-        for (int i = 0; i < nt; ++i) {
+        int issued = pre;
+        for (int i = pre; i < nt; ++i) {
           const int st = i % kStages;
           const uint32_t ph = (i / kStages) & 1;
           if (!mbar_wait(&s.empty[st], ph ^ 1, s.abort, status)) break;
@@ -316,11 +340,11 @@ int launch_one(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& q
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
   ProfScope ps(GATHER ? "rerank_score" : "score", st);
-  kern<<<grid, kThreads, kSmemBytes, st>>>(kmap, qmap, a.K, a.wsel, a.p->q_pos,
-                                          a.p->key_offsets, a.cand, a.k_cand, a.groups,
-                                          a.group_count, tps, a.q_lo, a.I, a.ld,
-                                          a.p->total_keys, status_ptr());
-  return cuda_fail(cudaGetLastError(), "score_kernel");
+  return cuda_fail(launch_pdl(kern, grid, dim3(kThreads), kSmemBytes, st, kmap, qmap, a.K,
+                              a.wsel, a.p->q_pos, a.p->key_offsets, a.cand, a.k_cand, a.groups,
+                              a.group_count, tps, a.q_lo, a.I, a.ld, a.p->total_keys,
+                              status_ptr()),
+                   "score_kernel");
 }
 
 template <bool GATHER>
@@ -352,19 +376,20 @@ int launch_score(const ScoreArgs& a, cudaStream_t st) {
   rc = make_kmajor_map(&qmap, a.qsel, (int64_t)a.p->num_queries * a.m, 32);
   if (rc) return rc;
   // Prefill-sized problems: about 8 CTAs per SM over the whole causal work,
-  // for balance.  Decode-sized problems (fewer groups than SMs): one wave, so
-  // that each CTA streams a long key range through its pipeline rather than
-  // paying its set-up for a few tiles in many waves.
+  // for balance.  Decode-sized problems (fewer groups than SMs): one wave of
+  // one CTA per SM, so that each CTA streams a long key range through its
+  // pipeline rather than paying its set-up for a few tiles in many waves;
+  // the device splits the wave among the groups that the plan produced.
   const int sms = num_sms();
-  int tps;
   if (a.max_groups < sms) {
-    const int splits = max(1, sms / a.max_groups);
-    tps = (a.max_tiles + splits - 1) / splits;
-  } else {
-    const int64_t work = (int64_t)a.max_groups * a.max_tiles;
-    tps = (int)((work + 8 * sms - 1) / (8 * sms));
-    tps = max(1, min(tps, 64));
+    // The device divides the SMs among the groups it finds (tiles_per_split 0).
+    dim3 grid(sms, 1);
+    return a.cand ? dispatch<true>(a, kmap, qmap, grid, 0, st)
+                  : dispatch<false>(a, kmap, qmap, grid, 0, st);
   }
+  const int64_t work = (int64_t)a.max_groups * a.max_tiles;
+  int tps = (int)((work + 8 * sms - 1) / (8 * sms));
+  tps = max(1, min(tps, 64));
   const int splits = (a.max_tiles + tps - 1) / tps;
   if (splits > 65535) {
     set_error("score: %d key splits exceed the grid limit", splits);

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
                 int n_fixed, const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
                 const int32_t* __restrict__ q_pos, int S, int q_lo, int k,
                 int32_t* __restrict__ idx_out, float* __restrict__ val_out, uint32_t* status) {
+  pdl_wait_then_release();
   __shared__ uint32_t hist[kMaxBins];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sel_bin, sel_above, sel_count, n_valid, out_cnt;
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
                         const int32_t* __restrict__ qo, const int32_t* __restrict__ q_pos, int S,
                         int q_lo, int k, int C, int32_t* __restrict__ idx_out,
                         float* __restrict__ val_out, uint32_t* status) {
+  pdl_wait_then_release();
   extern __shared__ __align__(16) uint64_t keys[];  // [kClusterCap]; 0 = not a candidate
   __shared__ uint32_t hist[2][kMaxBins];
   __shared__ uint32_t warp_tot[32];
@@ -405,13 +407,16 @@ int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the kernel waits on the previous one first
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     ProfScope ps("topk", st);
     cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, I, ld, tok, n_fixed,
                                        p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo,
@@ -419,10 +424,10 @@ int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32
     return cuda_fail(e, "topk_cluster_kernel");
   }
   ProfScope ps("topk", st);
-  topk_kernel<<<q_hi - q_lo, kTopkThreads, 0, st>>>(I, ld, tok, n_fixed, p.key_offsets,
-                                                    p.query_offsets, p.q_pos, p.num_seqs, q_lo,
-                                                    k, idx, val, status_ptr());
-  return cuda_fail(cudaGetLastError(), "topk_kernel");
+  return cuda_fail(launch_pdl(topk_kernel, dim3(q_hi - q_lo), dim3(kTopkThreads), 0, st, I, ld,
+                              tok, n_fixed, p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs,
+                              q_lo, k, idx, val, status_ptr()),
+                   "topk_kernel");
 }
 
 }  // namespace misa
