@@ -53,6 +53,8 @@ __global__ void block_offsets_kernel(const int64_t* __restrict__ ko, int S, int 
   }
 }
 
+constexpr int kSmallPlanGroups = 256;  // plans up to this many groups take one CTA
+
 // Query groups: every sequence's queries, restricted to [q_lo, q_hi), are cut
 // into groups of at most G, recorded as {seq, q_begin, q_end, max_pos}.
 // First a one-CTA scan over sequences gives each sequence the index of its
@@ -60,9 +62,9 @@ __global__ void block_offsets_kernel(const int64_t* __restrict__ ko, int S, int 
 // its sequence by binary search over first[] and reduces its queries'
 // positions.  Positions outside their sequence are flagged and left out of
 // max_pos.
-__global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_lo, int q_hi,
-                                  int G, int* __restrict__ first, int* __restrict__ count) {
-  pdl_wait_then_release();
+__device__ __forceinline__ void group_scan(const int32_t* __restrict__ qo, int S, int q_lo,
+                                           int q_hi, int G, int* __restrict__ first,
+                                           int* __restrict__ count) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
@@ -103,15 +105,19 @@ __global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_l
   if (threadIdx.x == 0) *count = carry;
 }
 
-__global__ void group_fill_kernel(const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
-                                  const int32_t* __restrict__ q_pos, int S, int q_lo, int q_hi,
-                                  int G, const int* __restrict__ first,
-                                  const int* __restrict__ count, int4* __restrict__ groups,
-                                  uint32_t* status) {
+__global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_lo, int q_hi,
+                                  int G, int* __restrict__ first, int* __restrict__ count) {
   pdl_wait_then_release();
+  group_scan(qo, S, q_lo, q_hi, G, first, count);
+}
+
+// Group fg (by one warp).
+__device__ __forceinline__ void group_fill(const int64_t* __restrict__ ko,
+                                           const int32_t* __restrict__ qo,
+                                           const int32_t* __restrict__ q_pos, int S, int q_lo,
+                                           int q_hi, int G, const int* __restrict__ first, int fg,
+                                           int4* __restrict__ groups, uint32_t* status) {
   const int lane = threadIdx.x & 31;
-  const int fg = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
-  if (fg >= *count) return;
   int lo = 0, hi = S - 1;  // last sequence j with first[j] <= fg
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -129,6 +135,34 @@ __global__ void group_fill_kernel(const int64_t* __restrict__ ko, const int32_t*
   }
   mp = __reduce_max_sync(0xffffffffu, mp);
   if (lane == 0) groups[fg] = make_int4(j, qb, qe, mp);
+}
+
+__global__ void group_fill_kernel(const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
+                                  const int32_t* __restrict__ q_pos, int S, int q_lo, int q_hi,
+                                  int G, const int* __restrict__ first,
+                                  const int* __restrict__ count, int4* __restrict__ groups,
+                                  uint32_t* status) {
+  pdl_wait_then_release();
+  const int fg = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
+  if (fg >= *count) return;
+  group_fill(ko, qo, q_pos, S, q_lo, q_hi, G, first, fg, groups, status);
+}
+
+// Both steps in one CTA, for plans of few groups (a decode batch): the scan,
+// a block barrier (the CTA's global writes are then visible to all its
+// threads), and the warps take the groups round-robin.
+__global__ void group_plan_small_kernel(const int64_t* __restrict__ ko,
+                                        const int32_t* __restrict__ qo,
+                                        const int32_t* __restrict__ q_pos, int S, int q_lo,
+                                        int q_hi, int G, int* __restrict__ first,
+                                        int* __restrict__ count, int4* __restrict__ groups,
+                                        uint32_t* status) {
+  pdl_wait_then_release();
+  group_scan(qo, S, q_lo, q_hi, G, first, count);
+  __syncthreads();
+  const int n = *count;
+  for (int fg = threadIdx.x >> 5; fg < n; fg += blockDim.x >> 5)
+    group_fill(ko, qo, q_pos, S, q_lo, q_hi, G, first, fg, groups, status);
 }
 
 // One warp per pooled row.  The two half-warps take alternate keys and each
@@ -226,12 +260,48 @@ __global__ void __launch_bounds__(256) pool_from_kernel(const uint16_t* __restri
     if (threadIdx.x == 0) set_status(status, MISA_STATUS_BOUNDS);
     return;
   }
-  for (int64_t b = f / B + warp; b < nblk; b += nw) {
+  const int64_t b0 = f / B;
+  if (nblk - b0 >= nw) {
+    for (int64_t b = b0 + warp; b < nblk; b += nw) {
+      const int64_t k0 = ko[s] + b * B;
+      const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
+      pool_row(K, k0, k1, bo[s] + b, Kbar);
+    }
+    return;
+  }
+  // Fewer new blocks than warps (a decode step): the whole CTA pools each
+  // block, 16 half-warps taking every 16th key, and the partial fp64 sums are
+  // added per dim through shared memory.  The fp64 sums are exact (see
+  // pool_row), so this split gives the same means as one warp per block.
+  __shared__ double part[16][kD];
+  const int hw = threadIdx.x >> 4, hl = lane & 15;
+  constexpr int kRow16 = kD / 8;
+  for (int64_t b = b0; b < nblk; ++b) {
     const int64_t k0 = ko[s] + b * B;
     const int64_t k1 = min(k0 + (int64_t)B, ko[s + 1]);
-    pool_row(K, k0, k1, bo[s] + b, Kbar);
+    const int64_t n = k1 - k0;
+    const uint4* src = reinterpret_cast<const uint4*>(K) + k0 * kRow16 + hl;
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    int64_t i = hw;
+    for (; i + 16 * 7 < n; i += 16 * 8) {  // keys i, i+16, ..., i+112
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (i + 16 * u) * kRow16);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add_bf16x8(acc, v[u]);
+    }
+    for (; i < n; i += 16) add_bf16x8(acc, __ldg(src + i * kRow16));
+    __syncthreads();  // the previous block's sums have been read
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part[hw][8 * hl + j] = acc[j];
+    __syncthreads();
+    if (threadIdx.x < kD) {
+      double t = 0.0;
+#pragma unroll
+      for (int h = 0; h < 16; ++h) t += part[h][threadIdx.x];
+      Kbar[(bo[s] + b) * kD + threadIdx.x] = __double2float_rn(t / (double)n);
+    }
   }
-  (void)lane;
 }
 
 }  // namespace
@@ -247,10 +317,16 @@ int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4*
                        int* count, cudaStream_t st) {
   ProfScope ps("plan_groups", st);
   int* first = count + 4;  // [S] after the count word (see groups_bytes)
+  const int64_t max_groups = (int64_t)(q_hi - q_lo + G - 1) / G + p.num_seqs;
+  if (max_groups <= kSmallPlanGroups) {
+    return cuda_fail(launch_pdl(group_plan_small_kernel, dim3(1), dim3(1024), 0, st,
+                                p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo, q_hi,
+                                G, first, count, groups, status_ptr()),
+                     "group_plan_small_kernel");
+  }
   cudaError_t e = launch_pdl(group_scan_kernel, dim3(1), dim3(1024), 0, st, p.query_offsets,
                              p.num_seqs, q_lo, q_hi, G, first, count);
   if (e != cudaSuccess) return cuda_fail(e, "group_scan_kernel");
-  const int64_t max_groups = (int64_t)(q_hi - q_lo + G - 1) / G + p.num_seqs;
   const int warps = 8;
   e = launch_pdl(group_fill_kernel, dim3((unsigned)((max_groups + warps - 1) / warps)),
                  dim3(warps * 32), 0, st, p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs,

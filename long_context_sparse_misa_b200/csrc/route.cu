@@ -22,6 +22,8 @@
 // partial block, and takes the top-m.  The number of ranges is taken on the
 // device from the actual group count, so that the (group, range) CTAs form
 // one wave.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -115,7 +117,30 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         reinterpret_cast<float4*>(kb)[i] = __ldg(kbar4 + (int64_t)c0 * (kD / 4) + i);
       __syncthreads();
       const int lim = min(nb, nfull - c0);
-      for (int b = 0; b < lim; ++b) {
+      // Two blocks at a time (independent chains); each block's dot product
+      // and the order of the ReLU sums are those of the one-block loop.
+      int b = 0;
+      for (; b + 1 < lim; b += 2) {
+        const float4* r0 = reinterpret_cast<const float4*>(kb + b * kD);
+        const float4* r1 = r0 + kD / 4;
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+        float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < kD / 4; i += 2) {
+          const float4 a = r0[i], c = r0[i + 1], a1 = r1[i], c1 = r1[i + 1];
+          ffma2(d0, d1, qreg[4 * i + 0], qreg[4 * i + 1], a.x, a.y);
+          ffma2(e0, e1, qreg[4 * i + 0], qreg[4 * i + 1], a1.x, a1.y);
+          ffma2(d0, d1, qreg[4 * i + 2], qreg[4 * i + 3], a.z, a.w);
+          ffma2(e0, e1, qreg[4 * i + 2], qreg[4 * i + 3], a1.z, a1.w);
+          ffma2(d2, d3, qreg[4 * i + 4], qreg[4 * i + 5], c.x, c.y);
+          ffma2(e2, e3, qreg[4 * i + 4], qreg[4 * i + 5], c1.x, c1.y);
+          ffma2(d2, d3, qreg[4 * i + 6], qreg[4 * i + 7], c.z, c.w);
+          ffma2(e2, e3, qreg[4 * i + 6], qreg[4 * i + 7], c1.z, c1.w);
+        }
+        acc += fmaxf((d0 + d1) + (d2 + d3), 0.f);
+        acc += fmaxf((e0 + e1) + (e2 + e3), 0.f);
+      }
+      for (; b < lim; ++b) {
         const float4* row = reinterpret_cast<const float4*>(kb + b * kD);
         float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
@@ -137,34 +162,57 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     __syncthreads();
     for (int i = tid; i < G * kD; i += kRouteThreads) part[i] = 0.f;
     __syncthreads();
-    // Thread per (query, pair of dims); keys summed in order, 8 loads in flight.
-    for (int item = tid; item < nq * (kD / 2); item += kRouteThreads) {
-      const int qi = item / (kD / 2), dp = item - qi * (kD / 2);
-      const int p2 = q_pos[qb + qi];
-      if (p2 < 0 || p2 >= L) continue;
-      const int f2 = (p2 + 1) / B * B;
-      const int cnt = p2 + 1 - f2;
-      if (cnt == 0) continue;
-      const uint32_t* col = reinterpret_cast<const uint32_t*>(K + (ko[seq] + f2) * kD) + dp;
+    // Queries whose partial blocks start at the same key share one staging of
+    // its rows: up to 64 rows (16 KB, the pooled-block stage) per round trip,
+    // then one thread per (query, pair of dims) adds its keys in order.
+    const uint16_t* Kseq = K + ko[seq] * kD;
+    uint16_t* rows = reinterpret_cast<uint16_t*>(kb);
+    constexpr int kStageRows = kChunk * kD * 4 / (kD * 2);  // 64 bf16 rows
+    int qi0 = 0;
+    while (qi0 < nq) {
+      // block-uniform: every thread reads the same positions
+      const int p0 = q_pos[qb + qi0];
+      const int f0 = (p0 + 1) / B * B;
+      if (p0 < 0 || p0 >= L || p0 + 1 == f0) {
+        ++qi0;
+        continue;
+      }
+      int qi1 = qi0 + 1, cmax = p0 + 1 - f0;
+      while (qi1 < nq && qi1 - qi0 < kRouteThreads / (kD / 2)) {  // <= 4 queries a pass
+        const int p1 = q_pos[qb + qi1];
+        if (p1 < 0 || p1 >= L || (p1 + 1) / B * B != f0) break;
+        cmax = max(cmax, p1 + 1 - f0);
+        ++qi1;
+      }
+      const int item = tid;  // (query qi0 + item / 64, dims 2*(item % 64) and +1)
+      const int qi = qi0 + item / (kD / 2), dp = item % (kD / 2);
+      int cnt = 0;
+      if (qi < qi1) {
+        const int p2 = q_pos[qb + qi];
+        cnt = p2 + 1 - f0;  // 0 when this query's block is complete
+        if (cnt < 0) cnt = 0;
+      }
       float s0 = 0.f, s1 = 0.f;
-      int key = 0;
-      for (; key + 8 <= cnt; key += 8) {
-        uint32_t v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldg(col + (int64_t)(key + u) * (kD / 2));
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          s0 += __uint_as_float(v[u] << 16);
-          s1 += __uint_as_float(v[u] & 0xFFFF0000u);
+      for (int c0 = 0; c0 < cmax; c0 += kStageRows) {
+        const int nr = min(kStageRows, cmax - c0);
+        __syncthreads();
+        const uint4* src = reinterpret_cast<const uint4*>(Kseq + (int64_t)(f0 + c0) * kD);
+        for (int i = tid; i < nr * (kD / 8); i += kRouteThreads)
+          reinterpret_cast<uint4*>(rows)[i] = __ldg(src + i);
+        __syncthreads();
+        const uint32_t* col = reinterpret_cast<const uint32_t*>(rows) + dp;
+        const int lim = min(cnt - c0, nr);
+        for (int key = 0; key < lim; ++key) {
+          const uint32_t v = col[key * (kD / 2)];
+          s0 += __uint_as_float(v << 16);
+          s1 += __uint_as_float(v & 0xFFFF0000u);
         }
       }
-      for (; key < cnt; ++key) {
-        const uint32_t v = __ldg(col + (int64_t)key * (kD / 2));
-        s0 += __uint_as_float(v << 16);
-        s1 += __uint_as_float(v & 0xFFFF0000u);
+      if (cnt > 0) {
+        part[qi * kD + 2 * dp] = s0 / (float)cnt;
+        part[qi * kD + 2 * dp + 1] = s1 / (float)cnt;
       }
-      part[qi * kD + 2 * dp] = s0 / (float)cnt;
-      part[qi * kD + 2 * dp + 1] = s1 / (float)cnt;
+      qi0 = qi1;
     }
     __syncthreads();
     if (valid && nfull * B != n) {
@@ -188,8 +236,16 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     return;
   }
   if (kMode == kFinish && valid) {
+    // the ns + 1 range sums, loaded 8 at a time and added in range order
     const float* pp = partial + (int64_t)g * slots * kRouteThreads + tid;
-    for (int j = 0; j <= ns; ++j) acc += pp[(int64_t)j * kRouteThreads];
+    for (int j0 = 0; j0 <= ns; j0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = j0 + u <= ns ? pp[(int64_t)(j0 + u) * kRouteThreads] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u <= ns) acc += v[u];
+    }
   }
 
   float r = -INFINITY;
@@ -271,10 +327,13 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
   if ((rc = set_smem_limit((const void*)route_kernel<kPartial>, smem))) return rc;
   if ((rc = set_smem_limit((const void*)route_kernel<kFinish>, smem))) return rc;
   {
-    // One CTA per (group, range) and one per group for its partial block;
-    // the device uses the first count * (ns + 1) of them.
+    // One CTA per (group, range) and one per group for its partial block:
+    // the device uses the first count * (ns + 1) of the grid, at most
+    // max(sms, 2 * count) since ns + 1 <= max(2, sms / count).
     ProfScope ps("route", st);
-    rc = cuda_fail(launch_pdl(route_kernel<kPartial>, dim3(max_groups * (nsplit + 1)),
+    const int ranged = (int)std::min<int64_t>((int64_t)max_groups * (nsplit + 1),
+                                              std::max(sms, 2 * max_groups));
+    rc = cuda_fail(launch_pdl(route_kernel<kPartial>, dim3(ranged),
                               dim3(kRouteThreads), smem, st, q, w, K, Kbar, p.key_offsets,
                               p.block_offsets, p.q_pos, groups, group_count, p.num_heads,
                               p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(),
