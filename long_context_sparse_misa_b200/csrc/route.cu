@@ -16,10 +16,11 @@
 //
 // Decode batches have too few query groups to fill the GPU, and each group
 // scans every pooled block of a long prefix.  There the pooled blocks are
-// split into contiguous ranges, one CTA per (group, range) writes its partial
-// sums, and a second launch adds the ranges in ascending order (a fixed
-// order, so the result does not depend on scheduling), adds the causal
-// partial block, and takes the top-m.  The number of ranges is taken on the
+// split into contiguous ranges: one CTA per (group, range), and one per group
+// for its queries' causal partial blocks, write per-slot partial sums
+// (route_mma_kernel, on warp-level tensor-core MMAs), and a second launch
+// adds them in range order (a fixed order, so the result does not depend on
+// scheduling) and takes the top-m.  The number of ranges is taken on the
 // device from the actual group count, so that the (group, range) CTAs form
 // one wave.
 #include <algorithm>
@@ -34,11 +35,10 @@ constexpr int kRouteThreads = 256;
 constexpr int kChunk = 32;  // pooled blocks per shared-memory stage
 
 // kWhole: one CTA does everything for its group.
-// kPartial: CTA (group, y) with y < ns sums range y of the full pooled
-//           blocks; CTA (group, ns) evaluates the causal partial block.  Each
-//           stores its per-thread sum; nothing else.
-// kFinish: adds the ns + 1 stored sums in order, then ranks as kWhole.
-enum RouteMode { kWhole = 0, kPartial = 1, kFinish = 2 };
+// kFinish: adds the ns + 1 per-slot sums that route_mma_kernel stored for the
+//          group (ranges y < ns of the full pooled blocks, then the causal
+//          partial block) in order, then ranks as kWhole.
+enum RouteMode { kWhole = 0, kFinish = 2 };
 
 template <int kMode>
 __global__ void __launch_bounds__(kRouteThreads, 1)
@@ -57,14 +57,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   float* rs = part + G * kD;                  // [G][H]
 
   const int count = *group_count;
-  // Full-block ranges per group (kPartial / kFinish): as many as keep the
-  // count * (ns + 1) CTAs within one wave.
+  // Full-block ranges per group (kFinish): as many as keep the
+  // count * (ns + 1) CTAs of the ranges launch within one wave.
   const int ns = kMode == kWhole ? 1 : max(1, min(nsplit_max, sms / max(count, 1) - 1));
-  const int g = kMode == kPartial ? (int)blockIdx.x / (ns + 1) : (int)blockIdx.x;
+  const int g = (int)blockIdx.x;
   if (g >= count) return;
-  const int y = kMode == kPartial ? (int)blockIdx.x - g * (ns + 1) : 0;
-  const bool do_full = kMode == kWhole || (kMode == kPartial && y < ns);
-  const bool do_tail = kMode == kWhole || (kMode == kPartial && y == ns);
+  const bool do_full = kMode == kWhole, do_tail = kMode == kWhole;
   const int4 grp = groups[g];
   const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
   const int tid = threadIdx.x;
@@ -99,16 +97,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     for (int i = 0; i < kD; ++i) qreg[i] = 0.f;
   }
 
-  // Full blocks: ReLU(q . Kbar_b) summed over b < nfull (over this CTA's
-  // range of blocks when split).
+  // Full blocks: ReLU(q . Kbar_b) summed over b < nfull.
   float acc = 0.f;
   if (do_full) {
-    int b_lo = 0, b_hi = max_full;
-    if (kMode == kPartial) {
-      const int range = (max_full + ns - 1) / ns;
-      b_lo = y * range;
-      b_hi = min(max_full, b_lo + range);
-    }
+    const int b_lo = 0, b_hi = max_full;
     const float4* kbar4 = reinterpret_cast<const float4*>(Kbar + bo[seq] * kD);
     for (int c0 = b_lo; c0 < b_hi; c0 += kChunk) {
       const int nb = min(kChunk, b_hi - c0);
@@ -231,10 +223,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   }
 
   const int64_t slots = nsplit_max + 1;  // stored sums per group
-  if (kMode == kPartial) {
-    partial[((int64_t)g * slots + y) * kRouteThreads + tid] = acc;
-    return;
-  }
   if (kMode == kFinish && valid) {
     // the ns + 1 range sums, loaded 8 at a time and added in range order
     const float* pp = partial + (int64_t)g * slots * kRouteThreads + tid;
@@ -287,6 +275,238 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- ranges on tensor cores
+// The ranges of a decode batch on warp-level tensor-core MMAs (mma.sync
+// m16n8k16, bf16 inputs, fp32 accumulation).  CTA (group, y): y < ns sums
+// range y of the full pooled blocks, y == ns the queries' causal partial
+// blocks.  Each warp takes 16 (query, head) slots (A = their q rows, exact in
+// bf16) against 8 pooled blocks at a time (B = Kbar as a bf16 pair hi + lo,
+// hi + lo ~= Kbar to about 2^-16 relative, so q . Kbar = q . hi + q . lo).
+// A CUDA-core loop with one thread per slot is bound by shared-memory operand
+// traffic (every thread reads every pooled row); the MMA reads each row once
+// per warp.  The ReLU sum over the range's blocks is taken on the
+// accumulator fragments and added across the 4 lanes of a row at the end; the
+// partial blocks are one more MMA against the group's partial means.  Stores
+// one sum per slot and range, which route_kernel<kFinish> adds up.
+constexpr int kMmaBlock = 512;              // 16 warps x 16 slots = kRouteThreads
+constexpr int kRowW = kD / 2 + 4;           // words per staged row: 64 bf16 pairs + 4 pad
+
+__device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+}
+
+// hi / lo bf16 pairs of two fp32 values: hi = bf16(x), lo = bf16(x - hi).
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+  const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+  hi = bf16_pair(h0, h1);
+  lo = bf16_pair(x0 - h0, x1 - h1);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// C = A (16 slots x 128 dims, fragments a[kk]) x B (128 dims x 8 rows of the
+// staged hi / lo arrays, starting at row r0), both halves of the pair.
+__device__ __forceinline__ void mma_rows(float (&c)[4], const uint32_t (&a)[kD / 16][4],
+                                         const uint32_t* hi, const uint32_t* lo, int r0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  c[0] = c[1] = c[2] = c[3] = 0.f;
+  const uint32_t* h = hi + (r0 + g) * kRowW + t;
+  const uint32_t* l = lo + (r0 + g) * kRowW + t;
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    mma_bf16_16816(c, a[kk], h[8 * kk], h[8 * kk + 4]);
+    mma_bf16_16816(c, a[kk], l[8 * kk], l[8 * kk + 4]);
+  }
+}
+
+__global__ void __launch_bounds__(kMmaBlock, 1)
+    route_mma_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ K,
+                     const float* __restrict__ Kbar, const int64_t* __restrict__ ko,
+                     const int64_t* __restrict__ bo, const int32_t* __restrict__ q_pos,
+                     const int4* __restrict__ groups, const int* __restrict__ group_count,
+                     int H, int B, int G, int nsplit_max, int sms, float* __restrict__ partial) {
+  pdl_wait_then_release();
+  extern __shared__ __align__(16) uint32_t smem_w[];
+  uint32_t* khi = smem_w;                          // [kChunk][kRowW]
+  uint32_t* klo = khi + kChunk * kRowW;            // [kChunk][kRowW]
+  float* part = reinterpret_cast<float*>(klo + kChunk * kRowW);  // [G][128]
+  const int G8 = (G + 7) / 8 * 8;
+  uint32_t* phi = reinterpret_cast<uint32_t*>(part + G * kD);     // [G8][kRowW]
+  uint32_t* plo = phi + G8 * kRowW;                               // [G8][kRowW]
+
+  const int count = *group_count;
+  const int ns = max(1, min(nsplit_max, sms / max(count, 1) - 1));
+  const int g_ = (int)blockIdx.x / (ns + 1);
+  if (g_ >= count) return;
+  const int y = (int)blockIdx.x - g_ * (ns + 1);
+  const int4 grp = groups[g_];
+  const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
+  const int64_t L = ko[seq + 1] - ko[seq];
+  const int max_full = (grp.w + 1) / B;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gi = lane >> 2, ti = lane & 3;
+
+  // This lane's two slots (rows gi and gi + 8 of the warp's 16) and their
+  // queries' full-block counts.
+  const int sA = warp * 16 + gi, sB = sA + 8;
+  int nA = 0, nB = 0, qA = -1, qB = -1;
+  {
+    const int a = sA / H, b = sB / H;
+    if (a < nq) {
+      const int p = q_pos[qb + a];
+      if (p >= 0 && p < L) { nA = p + 1; qA = a; }
+    }
+    if (b < nq) {
+      const int p = q_pos[qb + b];
+      if (p >= 0 && p < L) { nB = p + 1; qB = b; }
+    }
+  }
+  const int fA = nA / B, fB = nB / B;  // full blocks of the two slots' queries
+  const bool warp_active = warp * 16 < nq * H;
+  // A fragments: q rows of the warp's slots (zero rows for invalid slots).
+  uint32_t afr[kD / 16][4];
+  {
+    const uint32_t* rowA =
+        qA >= 0 ? reinterpret_cast<const uint32_t*>(q + ((int64_t)(qb + qA) * H + sA % H) * kD)
+                : nullptr;
+    const uint32_t* rowB =
+        qB >= 0 ? reinterpret_cast<const uint32_t*>(q + ((int64_t)(qb + qB) * H + sB % H) * kD)
+                : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      afr[kk][0] = rowA ? __ldg(rowA + 8 * kk + ti) : 0u;
+      afr[kk][1] = rowB ? __ldg(rowB + 8 * kk + ti) : 0u;
+      afr[kk][2] = rowA ? __ldg(rowA + 8 * kk + 4 + ti) : 0u;
+      afr[kk][3] = rowB ? __ldg(rowB + 8 * kk + 4 + ti) : 0u;
+    }
+  }
+  float accA = 0.f, accB = 0.f;  // this lane's share of its two slots' sums
+
+  if (y < ns) {
+    // ---- range y of the full blocks
+    const int range = (max_full + ns - 1) / ns;
+    const int b_lo = y * range, b_hi = min(max_full, b_lo + range);
+    const float2* kbar2 = reinterpret_cast<const float2*>(Kbar + bo[seq] * kD);
+    for (int c0 = b_lo; c0 < b_hi; c0 += kChunk) {
+      const int nb = min(kChunk, b_hi - c0);
+      __syncthreads();
+      for (int i = tid; i < kChunk * (kD / 2); i += kMmaBlock) {
+        const int r = i / (kD / 2), w = i - r * (kD / 2);
+        uint32_t hv = 0u, lv = 0u;
+        if (r < nb) {
+          const float2 x = __ldg(kbar2 + (int64_t)(c0 + r) * (kD / 2) + w);
+          split_pair(x.x, x.y, hv, lv);
+        }
+        khi[r * kRowW + w] = hv;
+        klo[r * kRowW + w] = lv;
+      }
+      __syncthreads();
+      if (warp_active) {
+        for (int nt = 0; nt * 8 < nb; ++nt) {
+          float c[4];
+          mma_rows(c, afr, khi, klo, nt * 8);
+          const int b0 = c0 + nt * 8 + 2 * ti;  // blocks of columns 2ti, 2ti + 1
+          accA += (b0 < fA ? fmaxf(c[0], 0.f) : 0.f) + (b0 + 1 < fA ? fmaxf(c[1], 0.f) : 0.f);
+          accB += (b0 < fB ? fmaxf(c[2], 0.f) : 0.f) + (b0 + 1 < fB ? fmaxf(c[3], 0.f) : 0.f);
+        }
+      }
+    }
+  } else {
+    // ---- the causal partial block of every query of the group
+    for (int i = tid; i < G * kD; i += kMmaBlock) part[i] = 0.f;
+    __syncthreads();
+    // Queries whose partial blocks start at the same key share one staging
+    // of its rows (64 rows per round trip, in the pooled-block stage); one
+    // thread per (query, pair of dims) adds its keys in order.
+    const uint16_t* Kseq = K + ko[seq] * kD;
+    uint16_t* rows = reinterpret_cast<uint16_t*>(khi);
+    constexpr int kStageRows = 64;  // 64 bf16 rows = 16 KB <= the two staged arrays
+    int qi0 = 0;
+    while (qi0 < nq) {
+      const int p0 = q_pos[qb + qi0];  // block-uniform
+      const int f0 = (p0 + 1) / B * B;
+      if (p0 < 0 || p0 >= L || p0 + 1 == f0) {
+        ++qi0;
+        continue;
+      }
+      int qi1 = qi0 + 1, cmax = p0 + 1 - f0;
+      while (qi1 < nq && qi1 - qi0 < kMmaBlock / (kD / 2)) {
+        const int p1 = q_pos[qb + qi1];
+        if (p1 < 0 || p1 >= L || (p1 + 1) / B * B != f0) break;
+        cmax = max(cmax, p1 + 1 - f0);
+        ++qi1;
+      }
+      const int qi = qi0 + tid / (kD / 2), dp = tid % (kD / 2);
+      int cnt = 0;
+      if (qi < qi1) cnt = max(0, q_pos[qb + qi] + 1 - f0);
+      float s0 = 0.f, s1 = 0.f;
+      for (int c0 = 0; c0 < cmax; c0 += kStageRows) {
+        const int nr = min(kStageRows, cmax - c0);
+        __syncthreads();
+        const uint4* src = reinterpret_cast<const uint4*>(Kseq + (int64_t)(f0 + c0) * kD);
+        for (int i = tid; i < nr * (kD / 8); i += kMmaBlock)
+          reinterpret_cast<uint4*>(rows)[i] = __ldg(src + i);
+        __syncthreads();
+        const uint32_t* col = reinterpret_cast<const uint32_t*>(rows) + dp;
+        const int lim = min(cnt - c0, nr);
+        for (int key = 0; key < lim; ++key) {
+          const uint32_t v = col[key * (kD / 2)];
+          s0 += __uint_as_float(v << 16);
+          s1 += __uint_as_float(v & 0xFFFF0000u);
+        }
+      }
+      if (cnt > 0) {
+        part[qi * kD + 2 * dp] = s0 / (float)cnt;
+        part[qi * kD + 2 * dp + 1] = s1 / (float)cnt;
+      }
+      qi0 = qi1;
+    }
+    __syncthreads();
+    for (int i = tid; i < G8 * (kD / 2); i += kMmaBlock) {
+      const int r = i / (kD / 2), w = i - r * (kD / 2);
+      uint32_t hv = 0u, lv = 0u;
+      if (r < G) split_pair(part[r * kD + 2 * w], part[r * kD + 2 * w + 1], hv, lv);
+      phi[r * kRowW + w] = hv;
+      plo[r * kRowW + w] = lv;
+    }
+    __syncthreads();
+    // C[slot, query row]: each slot takes the column of its own query, if
+    // that query has a partial block.
+    if (warp_active) {
+      for (int nt = 0; nt * 8 < G; ++nt) {
+        float c[4];
+        mma_rows(c, afr, phi, plo, nt * 8);
+        const int col0 = nt * 8 + 2 * ti;
+        const bool pa = qA >= 0 && fA * B != nA, pb = qB >= 0 && fB * B != nB;
+        if (pa && qA == col0) accA += fmaxf(c[0], 0.f);
+        if (pa && qA == col0 + 1) accA += fmaxf(c[1], 0.f);
+        if (pb && qB == col0) accB += fmaxf(c[2], 0.f);
+        if (pb && qB == col0 + 1) accB += fmaxf(c[3], 0.f);
+      }
+    }
+  }
+
+  // Add the 4 lanes of each row; lane ti == 0 stores the slot sums.
+  accA += __shfl_xor_sync(0xffffffffu, accA, 1);
+  accA += __shfl_xor_sync(0xffffffffu, accA, 2);
+  accB += __shfl_xor_sync(0xffffffffu, accB, 1);
+  accB += __shfl_xor_sync(0xffffffffu, accB, 2);
+  if (ti == 0) {
+    const int64_t base = ((int64_t)g_ * (nsplit_max + 1) + y) * kRouteThreads;
+    partial[base + sA] = accA;
+    partial[base + sB] = accB;
+  }
+}
+
 }  // namespace
 
 int route_group_size(int H) { return H >= kRouteThreads ? 1 : kRouteThreads / H; }
@@ -324,7 +544,6 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
                                 (float*)nullptr),
                      "route_kernel");
   }
-  if ((rc = set_smem_limit((const void*)route_kernel<kPartial>, smem))) return rc;
   if ((rc = set_smem_limit((const void*)route_kernel<kFinish>, smem))) return rc;
   {
     // One CTA per (group, range) and one per group for its partial block:
@@ -333,12 +552,14 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
     ProfScope ps("route", st);
     const int ranged = (int)std::min<int64_t>((int64_t)max_groups * (nsplit + 1),
                                               std::max(sms, 2 * max_groups));
-    rc = cuda_fail(launch_pdl(route_kernel<kPartial>, dim3(ranged),
-                              dim3(kRouteThreads), smem, st, q, w, K, Kbar, p.key_offsets,
-                              p.block_offsets, p.q_pos, groups, group_count, p.num_heads,
-                              p.block, m, G, heads, q_r, w_r, router_scores, status_ptr(),
-                              nsplit, sms, partial),
-                   "route_kernel (ranges)");
+    const int G8 = (G + 7) / 8 * 8;
+    const int msmem = (2 * kChunk * kRowW + 2 * G8 * kRowW) * (int)sizeof(uint32_t) +
+                      G * kD * (int)sizeof(float);
+    if ((rc = set_smem_limit((const void*)route_mma_kernel, msmem))) return rc;
+    rc = cuda_fail(launch_pdl(route_mma_kernel, dim3(ranged), dim3(kMmaBlock), msmem, st, q, K,
+                              Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups,
+                              group_count, p.num_heads, p.block, G, nsplit, sms, partial),
+                   "route_mma_kernel (ranges)");
     if (rc) return rc;
   }
   ProfScope ps("route_finish", st);
