@@ -54,7 +54,11 @@ def test_pool_keys_bit_exact(B):
 
 
 # ------------------------------------------------------------------ router
-@pytest.mark.parametrize("H,m,B", [(16, 4, 64), (64, 8, 64), (32, 8, 128), (8, 8, 16), (64, 1, 32)])
+# (16, 4, 32), (32, 8, 16), (8, 8, 16) and (64, 1, 32) have enough pooled blocks per
+# group to take the split path (tensor-core ranges, finish launch) with 16, 8, 32 and 4
+# queries per group; the others run one CTA per group.
+@pytest.mark.parametrize("H,m,B", [(16, 4, 64), (64, 8, 64), (32, 8, 128), (8, 8, 16), (64, 1, 32),
+                                   (16, 4, 32), (32, 8, 16)])
 def test_route_ragged(H, m, B):
     wl = ragged(seed=H + m, H=H, B=B, m=m)
     prob, K, q, w = dev(wl)
