@@ -256,7 +256,8 @@ struct StreamPlan {
   bool use = false;
   int G = 0, grid = 0, max_groups = 0;
   int64_t cap = 0;
-  size_t bytes = 0;
+  size_t bytes = 0;           // selection inside the scoring kernel
+  size_t bytes_deferred = 0;  // plus lists per query, selected by a second launch
 };
 
 StreamPlan stream_plan(const misa_problem_t* p, int m, int k, bool want_rows) {
@@ -271,6 +272,7 @@ StreamPlan stream_plan(const misa_problem_t* p, int m, int k, bool want_rows) {
   sp.cap = stream_subcap(p->max_seq_len);
   sp.bytes = groups_bytes(T, p->num_seqs) + fail_bytes(T) +
              align_up(stream_cand_bytes(sp.grid, sp.cap, m));
+  sp.bytes_deferred = sp.bytes + align_up(stream_deferred_bytes(T, sp.cap, k));
   sp.use = true;
   return sp;
 }
@@ -294,6 +296,15 @@ int score_topk_impl(const misa_problem_t* p, const uint16_t* qsel, const float* 
     a.fail_list = reinterpret_cast<int32_t*>(fb + 16);
     a.cand = reinterpret_cast<uint2*>(fb + fail_bytes(T));
     a.subcap = sp.cap; a.idx = idx; a.val = val;
+    if (ws_bytes >= sp.bytes_deferred) {
+      // lists per query after the in-kernel buffers: [T][drows][128], counts, anchors
+      uint8_t* db = reinterpret_cast<uint8_t*>(a.cand) + align_up(stream_cand_bytes(sp.grid, sp.cap, m));
+      a.drows = stream_deferred_rows(k, sp.cap);
+      a.dcand = reinterpret_cast<uint2*>(db);
+      const size_t lists = align_up((size_t)T * a.drows * 128 * sizeof(uint2));
+      a.dcnt = reinterpret_cast<int*>(db + lists);
+      a.danchor = reinterpret_cast<int*>(db + lists + align_up((size_t)T * 128 * sizeof(int)));
+    }
     return launch_score_stream(a, st);
   }
   const int64_t ld = scores_dbg ? scores_ld : row_ld(p);
@@ -392,7 +403,7 @@ size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_
   const int ks = k_cand > k ? k_cand : k;
   for (int mm : {m, p->num_heads}) {
     const StreamPlan sp = stream_plan(p, mm, ks, false);
-    if (sp.use && sp.bytes > need) need = sp.bytes;
+    if (sp.use && sp.bytes_deferred > need) need = sp.bytes_deferred;
   }
   return need;
 }

@@ -151,8 +151,16 @@ struct StreamArgs {
   float* val;
   int32_t* fail_list;     // [T] queries whose sampled threshold did not verify
   int* fail_count;        // device counter for fail_list
+  // Deferred selection (nullptr dcand: selection inside the scoring kernel):
+  // one list per query row, stream_deferred_bytes(T, subcap, k) in all.
+  uint2* dcand = nullptr;  // [T][drows][128]
+  int* dcnt = nullptr;     // [T][128]
+  int* danchor = nullptr;  // [T]
+  int drows = 0;           // stream_deferred_rows(k, subcap)
 };
 int launch_score_stream(const StreamArgs& a, cudaStream_t st);
+size_t stream_deferred_bytes(int T, int64_t subcap, int k);
+int stream_deferred_rows(int k, int64_t subcap);
 int stream_group_size(int m);
 size_t stream_cand_bytes(int grid, int64_t subcap, int m);
 int64_t stream_subcap(int max_seq_len);

@@ -457,11 +457,19 @@ __device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
 }
 
 // Candidate list of (buffer b, query slot q) of this CTA: rows_cap rows of 128.
+// Deferred selection (anchor != nullptr): one list per query row t instead,
+// [T][rows_cap][128] with counts [T][128] and the query's histogram anchor,
+// selected after the pass by select_deferred_kernel.
 struct Lists {
-  uint2* cand;   // [grid][2][slots][rows_cap][128]
-  int* cnt;      // [grid][2][slots][128]
+  uint2* cand;   // [grid][2][slots][rows_cap][128], or [T][rows_cap][128]
+  int* cnt;      // [grid][2][slots][128], or [T][128]
   int rows_cap;
   int slots;
+  int* anchor;   // [T] deferred selection; nullptr: selected in the kernel
+  __device__ __forceinline__ uint2* list_t(int64_t t) const {
+    return cand + t * rows_cap * 128;
+  }
+  __device__ __forceinline__ int* counts_t(int64_t t) const { return cnt + t * 128; }
   __device__ __forceinline__ int64_t id(int b, int q) const {
     return ((int64_t)blockIdx.x * 2 + b) * slots + q;
   }
@@ -558,6 +566,7 @@ __global__ void __maxnreg__(96)
   const int count = *sc.count;
   if ((int)blockIdx.x >= count) return;
   const bool probe = sc.fail_in == nullptr;   // the fixup launch scans without a probe
+  const bool deferred = ls.anchor != nullptr;  // lists per query, selected after the launch
 
   Smem s = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -683,7 +692,7 @@ __global__ void __maxnreg__(96)
       const int np = probe_tiles(probe, ntiles);
       const int64_t L = ko[seq + 1] - ko[seq];
       const int bsel = gl & 1;
-      if (gl >= 2) {
+      if (gl >= 2 && !deferred) {
         // The group two back used this candidate buffer: claim what the
         // selectors have not taken yet, then wait until all of it is done.
         // The probe histograms are free here and serve as select scratch.
@@ -711,7 +720,9 @@ __global__ void __maxnreg__(96)
       for (int i = et; i < G * kHistWords; i += kEpiThreads) s.hist[i] = 0u;
       // This lane's list of its warp's first query (row-major over the 128
       // lists of a query) and its append counts, one per query.
-      uint2* mylist = ls.list(bsel, 0) + (int64_t)(half * QH) * ls.rows_cap * 128 + lrow;
+      uint2* mylist = (deferred ? ls.list_t(qb + half * QH)
+                                : ls.list(bsel, 0) + (int64_t)(half * QH) * ls.rows_cap * 128) +
+                      lrow;
       const uint32_t qstride = 128u * static_cast<uint32_t>(ls.rows_cap);
       const int rows_cap = ls.rows_cap;
       int cnt[QH];
@@ -834,6 +845,19 @@ __global__ void __maxnreg__(96)
         }
       }
       if (!ok) break;
+      if (deferred) {
+        // Leave the group's counts and histogram anchors for the selection
+        // pass after this launch.
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq)
+          if (half * QH + qq < nq) ls.counts_t(qb + half * QH + qq)[lrow] = cnt[qq];
+        // (each half's lane-quarter-0 warp wrote these anchors itself)
+        if (quarter == 0 && lane < QH && half * QH + lane < nq)
+          ls.anchor[qb + half * QH + lane] = s.base[half * QH + lane];
+        ++gl;
+        if (!(ok = ep_barrier(s, ephase, status))) break;
+        continue;
+      }
       // Hand the group to the selectors: counts, and (warp 0 of the
       // epilogue) the per-query positions, rows and histogram anchors.
 #pragma unroll
@@ -856,7 +880,7 @@ __global__ void __maxnreg__(96)
     }
     // Help the selectors with the last groups (no more probing: the
     // histograms are free).
-    for (int j = gl >= 2 ? gl - 2 : 0; ok && j < gl; ++j)
+    for (int j = gl >= 2 ? gl - 2 : 0; ok && !deferred && j < gl; ++j)
       select_claimed(s, ls, sc, j & 1, s.selnq[j & 1], k, idx_out, val_out,
                      s.hist + e * kSelBins);
   } else {
@@ -866,7 +890,7 @@ __global__ void __maxnreg__(96)
     const int sw = warp - 2 - kEpiWarps;  // 0..kSelWarps-1
     uint32_t* selh = s.sel + sw * kSelBins;
     int gl = 0;
-    bool ok = true;
+    bool ok = !deferred;  // deferred selection: nothing to do here
     for (int j = 0, gs = blockIdx.x; ok && gs < count; gs = sched_slot(++j)) {
       const int4 grp = fetch_group(sc, count, gs);
       if (grp.w < 0) continue;
@@ -885,6 +909,94 @@ __global__ void __maxnreg__(96)
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+}
+
+// Deferred selection: one warp per query row, after the scoring launch.
+// The same check and exact selection as select_query, on the query's own
+// lists; queries that fail the check go to the rescan list.  The lists were
+// written long before and sit in DRAM, so each warp runs a short pipeline
+// over its queries t, t + nw, ...: the counts of the query two ahead are
+// loaded, and the rows of the next query are requested into L2 (bulk
+// prefetch, one 1 KB row of all 128 lists per request), while the current
+// query is selected.
+constexpr int kSelectThreads = 256;
+constexpr int kSelectCtasPerSm = 4;
+
+struct QCounts {
+  int c0, c1, c2, c3;
+};
+
+__device__ __forceinline__ QCounts load_counts(const Lists& ls, int t, int T) {
+  const int lane = threadIdx.x & 31;
+  QCounts c = {0, 0, 0, 0};
+  if (t < T) {
+    const int* q = ls.counts_t(t);
+    c.c0 = q[lane];
+    c.c1 = q[lane + 32];
+    c.c2 = q[lane + 64];
+    c.c3 = q[lane + 96];
+  }
+  return c;
+}
+
+__device__ __forceinline__ void prefetch_lists(const Lists& ls, int t, int T, const QCounts& c) {
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  int rows = __reduce_max_sync(0xffffffffu, max(max(c.c0, c.c1), max(c.c2, c.c3)));
+  rows = min(rows, ls.rows_cap);
+  for (int r = lane; r < rows; r += 32) prefetch_l2_bulk(ls.list_t(t) + (int64_t)r * 128, 1024u);
+}
+
+__global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm)
+    select_deferred_kernel(Lists ls, const int32_t* __restrict__ q_pos,
+                           const int32_t* __restrict__ qo, const int64_t* __restrict__ ko, int S,
+                           int T, int k, int32_t* __restrict__ idx_out,
+                           float* __restrict__ val_out, int32_t* __restrict__ fail_out,
+                           int* __restrict__ fail_count) {
+  pdl_wait_then_release();
+  __shared__ uint32_t selh_all[kSelectThreads / 32][kSelBins];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* selh = selh_all[warp];
+  const int nw = (int)gridDim.x * (kSelectThreads / 32);
+  int t = (int)blockIdx.x * (kSelectThreads / 32) + warp;
+  QCounts cur = load_counts(ls, t, T), next = load_counts(ls, t + nw, T);
+  prefetch_lists(ls, t, T, cur);
+  for (; t < T; t += nw) {
+    prefetch_lists(ls, t + nw, T, next);
+    const QCounts after = load_counts(ls, t + 2 * nw, T);
+    const int sq = upper_segment<int32_t>(qo, S, t);
+    const int64_t L = ko[sq + 1] - ko[sq];
+    const int p = q_pos[t];
+    int32_t* idx = idx_out + (int64_t)t * k;
+    float* val = val_out + (int64_t)t * k;
+    if (p < 0 || p >= L) {  // invalid position: padded row (the pass skipped it)
+      for (int j = lane; j < k; j += 32) {
+        idx[j] = -1;
+        val[j] = -INFINITY;
+      }
+    } else {
+      const int napp = __reduce_add_sync(0xffffffffu, cur.c0 + cur.c1 + cur.c2 + cur.c3);
+      const int cmax =
+          __reduce_max_sync(0xffffffffu, max(max(cur.c0, cur.c1), max(cur.c2, cur.c3)));
+      if (napp < min(k, p + 1) || cmax > ls.rows_cap) {
+        if (lane == 0) fail_out[atomicAdd(fail_count, 1)] = t;
+      } else {
+        final_select(ls.list_t(t), ls.counts_t(t), ls.anchor[t], k, idx, val, selh);
+      }
+    }
+    __syncwarp();
+    cur = next;
+    next = after;
+  }
+}
+
+// Rows of a deferred list: twice the expected candidates per lane (about
+// 1.4 k / 128 with the probe threshold) plus 16, within [32, 128] and no more
+// than one row per tile; a fuller list sends its query to the rescan.
+int deferred_rows(int k, int64_t rows_full) {
+  int64_t r = 2 * ((14 * (int64_t)k + 1279) / 1280) + 16;
+  r = r < 32 ? 32 : (r > kRowsCap ? kRowsCap : r);
+  return (int)(r < rows_full ? r : rows_full);
 }
 
 // Candidate storage (one workspace region, 256-byte aligned parts): the main
@@ -943,10 +1055,32 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
   fix_ls.cnt = reinterpret_cast<int*>(base + cl.main_lists + cl.main_counts + cl.fix_lists);
   fix_ls.rows_cap = cl.rows_full;
   fix_ls.slots = 1;
+  main_ls.anchor = fix_ls.anchor = nullptr;
   cudaError_t e = cudaMemsetAsync(a.fail_count, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "reset failure count");
-  int rc = launch_one<MH>(a, kmap, qmap, sc, main_ls, st);
-  if (rc) return rc;
+  int rc;
+  if (a.dcand) {
+    // Lists per query, selected by a second launch over all query rows.
+    Lists dl;
+    dl.cand = a.dcand;
+    dl.cnt = a.dcnt;
+    dl.rows_cap = a.drows;
+    dl.slots = 0;
+    dl.anchor = a.danchor;
+    if ((rc = launch_one<MH>(a, kmap, qmap, sc, dl, st))) return rc;
+    {
+      ProfScope ps("select", st);
+      const int grid = kSelectCtasPerSm * num_sms();  // one wave
+      rc = cuda_fail(launch_pdl(select_deferred_kernel, dim3(grid), dim3(kSelectThreads), 0, st,
+                                dl, a.p->q_pos, a.p->query_offsets, a.p->key_offsets,
+                                a.p->num_seqs, a.p->num_queries, a.k, a.idx, a.val,
+                                a.fail_list, a.fail_count),
+                     "select_deferred_kernel");
+      if (rc) return rc;
+    }
+  } else if ((rc = launch_one<MH>(a, kmap, qmap, sc, main_ls, st))) {
+    return rc;
+  }
   // Queries whose probe threshold did not verify: rescan without a probe,
   // one query per group, with lists that hold every key.
   Sched fx = sc;
@@ -969,6 +1103,14 @@ size_t stream_cand_bytes(int grid, int64_t subcap, int m) {
   const CandLayout c = cand_layout(grid, subcap, kN / m);
   return c.main_lists + c.main_counts + c.fix_lists + c.fix_counts;
 }
+
+size_t stream_deferred_bytes(int T, int64_t subcap, int k) {
+  const int rows = deferred_rows(k, subcap);
+  return align256((size_t)T * rows * 128 * sizeof(uint2)) + align256((size_t)T * 128 * sizeof(int)) +
+         align256((size_t)T * sizeof(int));
+}
+
+int stream_deferred_rows(int k, int64_t subcap) { return deferred_rows(k, subcap); }
 
 int launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   if (a.max_groups <= 0) return MISA_OK;

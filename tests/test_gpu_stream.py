@@ -92,6 +92,35 @@ def test_stream_matches_rows_and_oracle(H, m, B, k):
                            heads=heads[sel].cpu().numpy(), k=k, m=m).assert_ok()
 
 
+def test_stream_selection_after_the_pass_and_in_kernel_agree():
+    # The workspace misa_workspace_size reports holds candidate lists per query,
+    # selected by a launch after the scoring pass; a smaller one (down to the
+    # double-buffered lists) selects inside the scoring kernel.  Same top-k.
+    wl = make_workload(seq_lens=[10000], queries="all", H=32, B=128, m=8, k=512, seed=31)
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    misa.profile_enable(True)
+    ix.misa(q, w, K)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert "select" in prof and "topk" not in prof
+    di, dv = ix.idx.clone(), ix.val.clone()
+    small = ix.ws[: ix.ws.numel() - 256]
+    misa.profile_enable(True)
+    misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, K, wl.k, ix.idx, ix.val, small)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert "select" not in prof and "topk" not in prof and "score" in prof
+    same_sets(di, dv, ix.idx, ix.val)
+    invariants(wl, di)
+    rows = sample_rows(wl, 30)
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_misa_rows(wl, rows, di[sel].cpu().numpy(), dv[sel].cpu().numpy(),
+                           heads=ix.heads[sel].cpu().numpy(), k=wl.k, m=wl.m).assert_ok()
+
+
 def test_stream_dense_multi_sequence():
     wl = make_workload(seq_lens=[5000, 3000, 2700], queries="all", H=32, B=128, m=8, k=512,
                        seed=9)
