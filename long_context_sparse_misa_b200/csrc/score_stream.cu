@@ -913,12 +913,11 @@ __global__ void __maxnreg__(96)
 
 // Deferred selection: one warp per query row, after the scoring launch.
 // The same check and exact selection as select_query, on the query's own
-// lists; queries that fail the check go to the rescan list.  The lists were
-// written long before and sit in DRAM, so each warp runs a short pipeline
-// over its queries t, t + nw, ...: the counts of the query two ahead are
-// loaded, and the rows of the next query are requested into L2 (bulk
-// prefetch, one 1 KB row of all 128 lists per request), while the current
-// query is selected.
+// lists; queries that fail the check go to the rescan list.  Each warp takes
+// queries t, t + nw, ... and loads the counts of the query two ahead while
+// it selects the current one.  (Requesting the next query's lists into L2
+// ahead of time measured slower: with 32 warps per SM the lists in flight
+// exceed L2, and the prefetched rows were evicted before use.)
 constexpr int kSelectThreads = 256;
 constexpr int kSelectCtasPerSm = 4;
 
@@ -939,14 +938,6 @@ __device__ __forceinline__ QCounts load_counts(const Lists& ls, int t, int T) {
   return c;
 }
 
-__device__ __forceinline__ void prefetch_lists(const Lists& ls, int t, int T, const QCounts& c) {
-  if (t >= T) return;
-  const int lane = threadIdx.x & 31;
-  int rows = __reduce_max_sync(0xffffffffu, max(max(c.c0, c.c1), max(c.c2, c.c3)));
-  rows = min(rows, ls.rows_cap);
-  for (int r = lane; r < rows; r += 32) prefetch_l2_bulk(ls.list_t(t) + (int64_t)r * 128, 1024u);
-}
-
 __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm)
     select_deferred_kernel(Lists ls, const int32_t* __restrict__ q_pos,
                            const int32_t* __restrict__ qo, const int64_t* __restrict__ ko, int S,
@@ -960,9 +951,7 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm)
   const int nw = (int)gridDim.x * (kSelectThreads / 32);
   int t = (int)blockIdx.x * (kSelectThreads / 32) + warp;
   QCounts cur = load_counts(ls, t, T), next = load_counts(ls, t + nw, T);
-  prefetch_lists(ls, t, T, cur);
   for (; t < T; t += nw) {
-    prefetch_lists(ls, t + nw, T, next);
     const QCounts after = load_counts(ls, t + 2 * nw, T);
     const int sq = upper_segment<int32_t>(qo, S, t);
     const int64_t L = ko[sq + 1] - ko[sq];
