@@ -40,17 +40,20 @@
 //     hold kRowsCap rows; a fuller list stops storing and sends its query to
 //     the rescan.  A query's 128 lists are stored row by row, so that a row
 //     of all lists is 1 KB contiguous.
-//   * check and select, by two selector warps while the epilogue warps
-//     already stream the next group (the candidate lists are double
-//     buffered; when the selectors fall behind, the epilogue warps claim the
-//     remaining queries of the older buffer before reusing it): every key
-//     scoring at least tau_q was appended, so if at
-//     least min(k, n) keys were appended (and no list ran past its rows) the
-//     exact top-k is among them.  The selector then histograms the
+//   * check and select: every key scoring at least tau_q was appended, so
+//     if at least min(k, n) keys were appended (and no list ran past its
+//     rows) the exact top-k is among them.  A warp then histograms the
 //     candidates, takes those above the bin holding the k-th, and resolves
 //     that bin with a warp-level radix select over (score, lower index
-//     first).  A query that fails the check is listed and rescanned by a
-//     second launch without a probe, with lists of one row per tile.
+//     first).  By default the lists are kept per query row and a second
+//     launch (select_deferred_kernel) checks and selects every query after
+//     the pass, so no selection work holds up the tensor pipe.  With less
+//     workspace the lists are double buffered per CTA and two selector warps
+//     check and select each finished group while the epilogue warps stream
+//     the next (when the selectors fall behind, the epilogue warps claim the
+//     remaining queries of the older buffer before reusing it).  A query that
+//     fails the check is listed and rescanned by a last launch without a
+//     probe, with lists of one row per tile (selected inside that launch).
 #include "common.cuh"
 #include "internal.h"
 
