@@ -19,7 +19,8 @@
 // head weight, and a causal compare -- no shuffles and no [m x L] tensor.
 //
 // Roles: warp 0 producer, warp 1 TMEM owner + MMA issuer (one thread),
-// warps 2..5 epilogue (TMEM lane quarter = warp % 4).
+// warps 2..5 epilogue (TMEM lane quarter = warp % 4); in gather mode warps 6
+// and 7 are two more producers.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,6 +28,13 @@ namespace misa {
 namespace {
 
 constexpr int kThreads = 192;
+// Gather mode adds two producer warps (6 and 7): the copies of a tile are
+// issued by one warp, tiles go round-robin over the three producers.
+constexpr int kGatherThreads = 256;
+constexpr int kGatherProducers = 3;
+__host__ __device__ constexpr int threads_for(bool gather) {
+  return gather ? kGatherThreads : kThreads;
+}
 constexpr int kStages = 4;
 constexpr int kStageBytes = kTileKeys * kD * 2;          // 32 KB: two 16 KB 64-dim halves
 constexpr int kHalfBytes = kStageBytes / 2;
@@ -75,7 +83,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
 }
 
 template <int MH, bool GATHER>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(GATHER), 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                  const uint16_t* __restrict__ K, const float* __restrict__ wsel,
                  const int32_t* __restrict__ q_pos, const int64_t* __restrict__ ko,
@@ -151,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     // Per-column head weight and per-query causal limit / output row.
     for (int c = threadIdx.x - 64; c < kMaxN; c += 128) {
       const int qi = c / MH;
@@ -173,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp >= 6) {
+    // ------------------------------------------------------------ producer(s)
     if (!GATHER) {
       if (lane == 0) {
         int issued = pre;
@@ -196,10 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
       // Gather mode: rows K[key_base + cand[t, slot]] for the 128 slots of a
-      // tile; each lane copies 4 rows as 16-byte chunks into the swizzled layout.
+      // tile; each lane copies 4 rows as 16-byte chunks into the swizzled
+      // layout.  Producer p (warp 0, 6, 7) takes tiles p, p + 3, ...
       const int t = qb;
       const int pos = s.pos[0];
-      if (lane == 0) {
+      const int prod = warp == 0 ? 0 : warp - 5;
+      if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&qmap);
         mbar_arrive_expect_tx(s.qfull, 2u * NP * 128u);
         for (int h = 0; h < 2; ++h)
@@ -208,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         qb * MH + r0);
       }
       __syncwarp();
-      int pending = -1;  // tile whose copies are committed but not yet signalled
-      int i = 0;
-      for (; i < nt; ++i) {
+      // Each producer has one tile in flight: copy, wait for its copies,
+      // signal; the three producers overlap.
+      for (int i = prod; i < nt; i += kGatherProducers) {
         const int st = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
         if (!warp_wait(&s.empty[st], ph ^ 1, s.abort, status)) break;
@@ -230,18 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         cp_async_commit();
-        if (pending >= 0) {
-          cp_async_wait_group<1>();
-          fence_proxy_async_smem();
-          mbar_arrive(&s.full[pending % kStages]);
-        }
-        pending = i;
+        cp_async_wait_group<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(&s.full[st]);
       }
       cp_async_wait_group<0>();
-      if (pending >= 0) {
-        fence_proxy_async_smem();
-        mbar_arrive(&s.full[pending % kStages]);
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -340,7 +343,7 @@ int launch_one(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& q
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
   ProfScope ps(GATHER ? "rerank_score" : "score", st);
-  return cuda_fail(launch_pdl(kern, grid, dim3(kThreads), kSmemBytes, st, kmap, qmap, a.K,
+  return cuda_fail(launch_pdl(kern, grid, dim3(threads_for(GATHER)), kSmemBytes, st, kmap, qmap, a.K,
                               a.wsel, a.p->q_pos, a.p->key_offsets, a.cand, a.k_cand, a.groups,
                               a.group_count, tps, a.q_lo, a.I, a.ld, a.p->total_keys,
                               status_ptr()),
