@@ -243,25 +243,26 @@ def workload_config(wl, cfg):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(wl, budget_s, seed=0):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_rows(wl, budget_s, seed, Kf, Kbar, boff):
+    """Oracle MISA (and re-rank) on random query rows until budget_s of work."""
     import numpy as np
     import oracle
-    try:
-        import threadpoolctl
-        cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
-    except Exception:
-        cores = 1
-    Kf = oracle.widen_bf16(wl.K_bits)
-    t0 = time.perf_counter()
-    Kbar = oracle.pool_keys(Kf, wl.key_offsets, wl.B)
-    t_pool = time.perf_counter() - t0
-    boff = oracle.block_offsets(wl.key_offsets, wl.B)
-    rng = np.random.default_rng(seed)
-    order = rng.permutation(wl.T)
-    qs = wl.q_seq
+    order = np.random.default_rng(seed).permutation(wl.T)
     pairs, rows, t_rows = 0, 0, 0.0
     for i in order:
-        s = int(qs[i])
+        s = int(wl.q_seq[i])
         k0, k1 = int(wl.key_offsets[s]), int(wl.key_offsets[s + 1])
         t1 = time.perf_counter()
         res = oracle.misa_query(oracle.widen_bf16(wl.q_bits[i]), wl.w[i].astype(np.float64),
@@ -275,11 +276,40 @@ def cpu_oracle_sample(wl, budget_s, seed=0):
         rows += 1
         if t_rows > budget_s:
             break
+    return pairs, rows, t_rows
+
+
+def cpu_oracle_sample(wl, budget_s, seed=0, one_core_s=0.0):
+    """The CPU oracle (numpy fp64, BLAS on all host cores) on a bounded
+    random sample of the workload's query rows, pooling charged pro rata;
+    with one_core_s > 0 also a shorter sample limited to one thread."""
+    import oracle
+    try:
+        import threadpoolctl
+        cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
+    except Exception:
+        threadpoolctl, cores = None, 1
+    Kf = oracle.widen_bf16(wl.K_bits)
+    t0 = time.perf_counter()
+    Kbar = oracle.pool_keys(Kf, wl.key_offsets, wl.B)
+    t_pool = time.perf_counter() - t0
+    boff = oracle.block_offsets(wl.key_offsets, wl.B)
+    pairs, rows, t_rows = _oracle_rows(wl, budget_s, seed, Kf, Kbar, boff)
     # pooling is per step; charge the sample its share
     t = t_rows + t_pool * pairs / max(wl.pairs, 1)
-    return {"value": pairs / t, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {wl.T} query rows (random, seed {seed}), {pairs} pairs, "
-                      f"{t:.2f} s incl. pro-rated pooling; numpy fp64"}
+    out = {"value": pairs / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": f"{rows} of {wl.T} query rows (random, seed {seed}), {pairs} pairs, "
+                     f"{t:.2f} s incl. pro-rated pooling; numpy fp64"}
+    if one_core_s > 0 and threadpoolctl is not None:
+        with threadpoolctl.threadpool_limits(1):
+            t0 = time.perf_counter()
+            oracle.pool_keys(Kf, wl.key_offsets, wl.B)
+            t_pool1 = time.perf_counter() - t0
+            p1, r1, t1 = _oracle_rows(wl, one_core_s, seed + 1, Kf, Kbar, boff)
+        out["value_1core"] = p1 / (t1 + t_pool1 * p1 / max(wl.pairs, 1))
+        out["sample_1core"] = f"{r1} query rows, {p1} pairs, {t1:.2f} s on one thread"
+    return out
 
 
 # ------------------------------------------------------------------ reference arm
@@ -601,7 +631,8 @@ def run_ours(args):
 
     # ---- CPU oracle on this host, rank 0 at N=1
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(wl, args.cpu_budget_s)
+        line["cpu_baseline"] = cpu_oracle_sample(wl, args.cpu_budget_s,
+                                                   one_core_s=args.cpu_budget_s / 4)
 
     if rank == 0:
         print(json.dumps(line), flush=True)
