@@ -434,15 +434,19 @@ def run_ours(args):
     # only) runs between steps, outside the timed intervals.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    step_prof = []  # per step: {kernel: (ms, launches)}
     for e0, e1 in evs:
         settle()
         e0.record()
         run()
         e1.record()
+        if graph is None:
+            # waits for this step's events (the next step's own events are
+            # recorded after the L2 flush and the device sleep)
+            step_prof.append(misa.profile_collect())
     torch.cuda.synchronize()
     clocks.end()
     clk = clocks.stop()
-    prof = misa.profile_collect()
     misa.profile_enable(False)
     barrier(world)
     step_ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
@@ -457,9 +461,14 @@ def run_ours(args):
         for _ in range(args.steps):
             settle()
             eager_run()
+            step_prof.append(misa.profile_collect())
         torch.cuda.synchronize()
-        prof = misa.profile_collect()
         misa.profile_enable(False)
+    prof = {}
+    for sp in step_prof:
+        for n, (t, c) in sp.items():
+            t0, c0 = prof.get(n, (0.0, 0))
+            prof[n] = (t0 + t, c0 + c)
     code, bits = misa.stream_status()
     if code != 0:
         raise RuntimeError(f"device status {code} ({bits}) in the timed region")
@@ -503,9 +512,16 @@ def run_ours(args):
                     "algorithmic_bytes_per_launch": abytes / max(launches_per_step, 1)}
     roofline |= {"launches_per_step": launches_per_step,
                  "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
-    kernels = {n: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps,
-                   "share": t / max(sum(v[0] for v in prof.values()), 1e-9)}
-               for n, (t, c) in prof.items()}
+    def pct(vals, q):
+        vals = sorted(vals)
+        return vals[min(len(vals) - 1, (q * len(vals)) // 100)]
+
+    kernels = {}
+    for n, (t, c) in prof.items():
+        per_step = [sp.get(n, (0.0, 0))[0] for sp in step_prof]
+        kernels[n] = {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps,
+                      "share": t / max(sum(v[0] for v in prof.values()), 1e-9),
+                      "p50_ms": pct(per_step, 50), "p90_ms": pct(per_step, 90)}
     gpu_launches = sum(c for _, c in prof.values())
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
