@@ -87,7 +87,13 @@ typedef struct {
 
 /* Bytes of workspace that any entry point below needs for this problem with
  * m routed heads, final top-k `k` and MISA-dagger candidate count `k_cand`
- * (0 if unused).  Returns 0 on invalid arguments. */
+ * (0 if unused), on its fastest path.  Returns 0 on invalid arguments.
+ * For a prefill that streams (misa_score_topk, dsa_index_dense) this
+ * includes candidate lists per query row for the exact selection after the
+ * scoring pass, about T * (2 * 1.4 * k / 128 + 16) KB (8.1 GB for 131072
+ * queries at k = 2048); a smaller workspace takes slower paths (selection
+ * inside the scoring kernel, then score rows with a separate top-k) and
+ * MISA_ERR_WORKSPACE_TOO_SMALL only below what the slowest path needs. */
 size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_t k_cand);
 
 /* block_offsets[s] = sum_{s'<s} ceil(L_s' / block) from key_offsets
