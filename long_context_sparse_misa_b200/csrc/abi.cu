@@ -555,10 +555,11 @@ int misa_hier_rerank(const misa_problem_t* p, const uint16_t* q, const float* w,
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve c = carve(ws, T, S);
-  if ((rc = launch_plan_groups(*p, 0, T, 1, c.groups, c.count, st))) return rc;
+  // one query per group: the scoring kernel takes query rows directly (no plan)
   ScoreArgs a;
   a.p = p; a.qsel = q; a.wsel = w; a.m = p->num_heads; a.K = K; a.cand = cand;
-  a.k_cand = k_cand; a.groups = c.groups; a.group_count = c.count; a.max_groups = T + S;
+  a.k_cand = k_cand; a.groups = nullptr; a.group_count = nullptr; a.max_groups = T;
+  a.direct = true;
   a.G = 1; a.q_lo = 0; a.I = c.buf; a.ld = k_cand;
   a.max_tiles = (k_cand + kTileKeys - 1) / kTileKeys;
   if ((rc = launch_score(a, st))) return rc;

@@ -130,6 +130,7 @@ struct ScoreArgs {
   float* I;               // output rows
   int64_t ld;
   int max_tiles;          // host bound on key tiles per group
+  bool direct = false;    // gather mode without a plan: group i is query row i
 };
 int launch_score(const ScoreArgs& a, cudaStream_t st);
 

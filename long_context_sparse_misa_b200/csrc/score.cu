@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
                  const int32_t* __restrict__ q_pos, const int64_t* __restrict__ ko,
                  const int32_t* __restrict__ cand, int k_cand, const int4* __restrict__ groups,
                  const int* __restrict__ group_count, int tiles_per_split, int q_lo,
-                 float* __restrict__ I, int64_t ld, int64_t total_keys, uint32_t* status) {
+                 float* __restrict__ I, int64_t ld, int64_t total_keys, uint32_t* status,
+                 const int32_t* __restrict__ qo, int S, int direct_T) {
   pdl_wait_then_release();
   constexpr int G = GATHER ? 1 : kMaxN / MH;
   static_assert(G * MH <= kMaxN, "group too wide");
@@ -98,7 +99,8 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
   // tiles_per_split > 0: CTA (x, y) takes group x, tiles from y * tiles_per_split.
   // tiles_per_split == 0: one wave of gridDim.x CTAs spread over the groups
   // that exist, gridDim.x / count consecutive CTAs per group.
-  const int count = *group_count;
+  // direct_T > 0 (gather mode): no group table; group i is query row i.
+  const int count = direct_T > 0 ? direct_T : *group_count;
   int gi = blockIdx.x, split = blockIdx.y, nsplit = 0;
   if (tiles_per_split == 0) {
     nsplit = count > 0 ? max(1, (int)gridDim.x / count) : 1;
@@ -106,7 +108,19 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
     split = blockIdx.x % nsplit;
   }
   if (gi >= count) return;
-  const int4 grp = groups[gi];
+  int4 grp;
+  if (GATHER && direct_T > 0) {
+    const int sq = upper_segment<int32_t>(qo, S, gi);
+    const int64_t Lq = ko[sq + 1] - ko[sq];
+    int pq = q_pos[gi];
+    if (pq < 0 || pq >= Lq) {  // as the planner: flagged, and the row is left out
+      if (split == 0 && threadIdx.x == 0) set_status(status, MISA_STATUS_BAD_INPUT);
+      pq = -1;
+    }
+    grp = make_int4(sq, gi, gi + 1, pq);
+  } else {
+    grp = groups[gi];
+  }
   const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y, maxpos = grp.w;
   if (maxpos < 0 || nq <= 0) return;
   const int64_t key_base = ko[seq];
@@ -346,7 +360,8 @@ int launch_one(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& q
   return cuda_fail(launch_pdl(kern, grid, dim3(threads_for(GATHER)), kSmemBytes, st, kmap, qmap, a.K,
                               a.wsel, a.p->q_pos, a.p->key_offsets, a.cand, a.k_cand, a.groups,
                               a.group_count, tps, a.q_lo, a.I, a.ld, a.p->total_keys,
-                              status_ptr()),
+                              status_ptr(), a.p->query_offsets, a.p->num_seqs,
+                              a.direct ? a.p->num_queries : 0),
                    "score_kernel");
 }
 
