@@ -478,7 +478,10 @@ int misa_route(const misa_problem_t* p, const uint16_t* q, const float* w, const
   // Split the block ranges only when the workspace holds the partial sums.
   int nsplit = route_split_count(*p, mg, num_sms());
   if (nsplit > 1 && ws_bytes < route_bytes(p)) nsplit = 1;
-  if ((rc = launch_plan_groups(*p, 0, T, G, c.groups, c.count, st))) return rc;
+  // the plan also clears the split path's per-group completion counters
+  int* done = nsplit > 1 ? route_split_counters(c.buf, mg, nsplit) : nullptr;
+  if ((rc = launch_plan_groups(*p, 0, T, G, c.groups, c.count, st, done, done ? mg : 0)))
+    return rc;
   return launch_route(*p, q, w, K, Kbar, m, heads, q_r, w_r, router_scores, c.groups, c.count,
                       mg, G, nsplit, nsplit > 1 ? c.buf : nullptr, st);
 }

@@ -70,8 +70,10 @@ int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* bloc
 // Build query groups of at most G queries over query rows [q_lo, q_hi).
 // groups: int4 [q_hi-q_lo + S]; count: one int, followed 16 bytes later by
 // int [S] of scratch (the first group of each sequence).
+// zero / nzero: an int array that the plan also clears (the router's
+// per-group completion counters), or nullptr.
 int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
-                       int* count, cudaStream_t st);
+                       int* count, cudaStream_t st, int* zero = nullptr, int nzero = 0);
 int launch_pool(const misa_problem_t& p, const uint16_t* K, float* Kbar, cudaStream_t st);
 // Re-pool only the blocks of each sequence s that hold keys >= from_pos[s].
 int launch_pool_from(const misa_problem_t& p, const uint16_t* K, float* Kbar,
@@ -87,6 +89,8 @@ int route_group_size(int H);
 // the workspace its partial sums take.
 int route_split_count(const misa_problem_t& p, int max_groups, int sms);
 size_t route_split_bytes(int max_groups, int nsplit);
+// The per-group completion counters inside that scratch (cleared by the plan).
+int* route_split_counters(float* partial, int max_groups, int nsplit);
 
 // ---- route_tc.cu: the router as a tcgen05 GEMM (prefill-sized problems).
 struct RouteTcArgs {

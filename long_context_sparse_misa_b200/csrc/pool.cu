@@ -106,8 +106,10 @@ __device__ __forceinline__ void group_scan(const int32_t* __restrict__ qo, int S
 }
 
 __global__ void group_scan_kernel(const int32_t* __restrict__ qo, int S, int q_lo, int q_hi,
-                                  int G, int* __restrict__ first, int* __restrict__ count) {
+                                  int G, int* __restrict__ first, int* __restrict__ count,
+                                  int* __restrict__ zero, int nzero) {
   pdl_wait_then_release();
+  for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   group_scan(qo, S, q_lo, q_hi, G, first, count);
 }
 
@@ -156,13 +158,19 @@ __global__ void group_plan_small_kernel(const int64_t* __restrict__ ko,
                                         const int32_t* __restrict__ q_pos, int S, int q_lo,
                                         int q_hi, int G, int* __restrict__ first,
                                         int* __restrict__ count, int4* __restrict__ groups,
-                                        uint32_t* status) {
+                                        uint32_t* status, int* __restrict__ zero, int nzero) {
   pdl_wait_then_release();
+  for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   group_scan(qo, S, q_lo, q_hi, G, first, count);
+  __syncthreads();
+  // S <= kSmallPlanGroups here: the first groups of the sequences go to
+  // shared memory for the warps' binary searches
+  __shared__ int sfirst[kSmallPlanGroups];
+  for (int s = threadIdx.x; s < S; s += blockDim.x) sfirst[s] = first[s];
   __syncthreads();
   const int n = *count;
   for (int fg = threadIdx.x >> 5; fg < n; fg += blockDim.x >> 5)
-    group_fill(ko, qo, q_pos, S, q_lo, q_hi, G, first, fg, groups, status);
+    group_fill(ko, qo, q_pos, S, q_lo, q_hi, G, sfirst, fg, groups, status);
 }
 
 // One warp per pooled row.  The two half-warps take alternate keys and each
@@ -314,18 +322,18 @@ int launch_block_offsets(const int64_t* key_offsets, int S, int B, int64_t* bloc
 }
 
 int launch_plan_groups(const misa_problem_t& p, int q_lo, int q_hi, int G, int4* groups,
-                       int* count, cudaStream_t st) {
+                       int* count, cudaStream_t st, int* zero, int nzero) {
   ProfScope ps("plan_groups", st);
   int* first = count + 4;  // [S] after the count word (see groups_bytes)
   const int64_t max_groups = (int64_t)(q_hi - q_lo + G - 1) / G + p.num_seqs;
   if (max_groups <= kSmallPlanGroups) {
     return cuda_fail(launch_pdl(group_plan_small_kernel, dim3(1), dim3(1024), 0, st,
                                 p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo, q_hi,
-                                G, first, count, groups, status_ptr()),
+                                G, first, count, groups, status_ptr(), zero, nzero),
                      "group_plan_small_kernel");
   }
   cudaError_t e = launch_pdl(group_scan_kernel, dim3(1), dim3(1024), 0, st, p.query_offsets,
-                             p.num_seqs, q_lo, q_hi, G, first, count);
+                             p.num_seqs, q_lo, q_hi, G, first, count, zero, nzero);
   if (e != cudaSuccess) return cuda_fail(e, "group_scan_kernel");
   const int warps = 8;
   e = launch_pdl(group_fill_kernel, dim3((unsigned)((max_groups + warps - 1) / warps)),

@@ -34,13 +34,8 @@ namespace {
 constexpr int kRouteThreads = 256;
 constexpr int kChunk = 32;  // pooled blocks per shared-memory stage
 
-// kWhole: one CTA does everything for its group.
-// kFinish: adds the ns + 1 per-slot sums that route_mma_kernel stored for the
-//          group (ranges y < ns of the full pooled blocks, then the causal
-//          partial block) in order, then ranks as kWhole.
-enum RouteMode { kWhole = 0, kFinish = 2 };
-
-template <int kMode>
+// One CTA per query group does everything for it (problems whose groups fill
+// the GPU, or without the scratch of the split path).
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w,
                  const uint16_t* __restrict__ K, const float* __restrict__ Kbar,
@@ -48,8 +43,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
                  const int32_t* __restrict__ q_pos, const int4* __restrict__ groups,
                  const int* __restrict__ group_count, int H, int B, int m, int G,
                  int32_t* __restrict__ heads, uint16_t* __restrict__ q_r, float* __restrict__ w_r,
-                 float* __restrict__ router_scores, uint32_t* status, int nsplit_max,
-                 int sms, float* __restrict__ partial) {
+                 float* __restrict__ router_scores, uint32_t* status) {
   pdl_wait_then_release();
   extern __shared__ __align__(16) float smem_f[];
   float* kb = smem_f;                         // [kChunk][128]
@@ -57,12 +51,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   float* rs = part + G * kD;                  // [G][H]
 
   const int count = *group_count;
-  // Full-block ranges per group (kFinish): as many as keep the
-  // count * (ns + 1) CTAs of the ranges launch within one wave.
-  const int ns = kMode == kWhole ? 1 : max(1, min(nsplit_max, sms / max(count, 1) - 1));
   const int g = (int)blockIdx.x;
   if (g >= count) return;
-  const bool do_full = kMode == kWhole, do_tail = kMode == kWhole;
+  constexpr bool do_full = true, do_tail = true;
   const int4 grp = groups[g];
   const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
   const int tid = threadIdx.x;
@@ -78,7 +69,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   const int max_full = (grp.w + 1) / B;
 
   float qreg[kD];
-  if (valid && kMode != kFinish) {
+  if (valid) {
     const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)t * H + h) * kD);
 #pragma unroll
     for (int i = 0; i < kD / 8; ++i) {
@@ -222,20 +213,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
   }
 
-  const int64_t slots = nsplit_max + 1;  // stored sums per group
-  if (kMode == kFinish && valid) {
-    // the ns + 1 range sums, loaded 8 at a time and added in range order
-    const float* pp = partial + (int64_t)g * slots * kRouteThreads + tid;
-    for (int j0 = 0; j0 <= ns; j0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = j0 + u <= ns ? pp[(int64_t)(j0 + u) * kRouteThreads] : 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (j0 + u <= ns) acc += v[u];
-    }
-  }
-
   float r = -INFINITY;
   if (valid) {
     const float wt = __ldg(w + (int64_t)t * H + h);
@@ -286,8 +263,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 // traffic (every thread reads every pooled row); the MMA reads each row once
 // per warp.  The ReLU sum over the range's blocks is taken on the
 // accumulator fragments and added across the 4 lanes of a row at the end; the
-// partial blocks are one more MMA against the group's partial means.  Stores
-// one sum per slot and range, which route_kernel<kFinish> adds up.
+// partial blocks are one more MMA against the group's partial means.  Each
+// CTA stores one sum per slot; the group's last CTA adds them in range order
+// and ranks the heads.
 constexpr int kMmaBlock = 512;              // 16 warps x 16 slots = kRouteThreads
 constexpr int kRowW = kD / 2 + 4;           // words per staged row: 64 bf16 pairs + 4 pad
 
@@ -333,7 +311,11 @@ __global__ void __launch_bounds__(kMmaBlock, 1)
                      const float* __restrict__ Kbar, const int64_t* __restrict__ ko,
                      const int64_t* __restrict__ bo, const int32_t* __restrict__ q_pos,
                      const int4* __restrict__ groups, const int* __restrict__ group_count,
-                     int H, int B, int G, int nsplit_max, int sms, float* __restrict__ partial) {
+                     int H, int B, int G, int nsplit_max, int sms, float* __restrict__ partial,
+                     int* __restrict__ done, const float* __restrict__ w, int m,
+                     int32_t* __restrict__ heads, uint16_t* __restrict__ q_r,
+                     float* __restrict__ w_r, float* __restrict__ router_scores,
+                     uint32_t* status) {
   pdl_wait_then_release();
   extern __shared__ __align__(16) uint32_t smem_w[];
   uint32_t* khi = smem_w;                          // [kChunk][kRowW]
@@ -505,6 +487,69 @@ __global__ void __launch_bounds__(kMmaBlock, 1)
     partial[base + sA] = accA;
     partial[base + sB] = accB;
   }
+
+  // The last of the group's ns + 1 CTAs to get here adds the stored sums in
+  // range order and ranks the group's heads (the counters are cleared by
+  // the plan launch before this one).
+  __shared__ int s_last;
+  __threadfence();  // this CTA's sums are visible before it counts itself
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&done[g_], 1) == ns;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* rs = reinterpret_cast<float*>(plo + G8 * kRowW);  // [G][H] router scores
+  const int slot = tid, qq = slot / H, h = slot - qq * H;
+  const bool active = slot < kRouteThreads && qq < nq;
+  const int t = qb + qq;
+  int pos = active ? q_pos[t] : -1;
+  const bool valid = active && pos >= 0 && pos < L;
+  float r = -INFINITY;
+  if (valid) {
+    float acc = 0.f;
+    const float* pp = partial + (int64_t)g_ * (nsplit_max + 1) * kRouteThreads + slot;
+    for (int j0 = 0; j0 <= ns; j0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = j0 + u <= ns ? __ldcg(pp + (int64_t)(j0 + u) * kRouteThreads) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u <= ns) acc += v[u];
+    }
+    r = __ldg(w + (int64_t)t * H + h) * acc;
+    if (router_scores) router_scores[(int64_t)t * H + h] = r;
+    if (r != r) {
+      set_status(status, MISA_STATUS_BAD_INPUT);
+      r = -INFINITY;
+    }
+  }
+  if (active) rs[qq * H + h] = r;
+  __syncthreads();
+  if (!active) return;
+  // Top-m by (r desc, head asc): rank of this head among the query's heads.
+  if (!valid) {
+    if (h < m) {  // invalid query: deterministic padding
+      heads[(int64_t)t * m + h] = -1;
+      w_r[(int64_t)t * m + h] = 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(q_r + ((int64_t)t * m + h) * kD);
+      for (int i = 0; i < kD / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+  int rank = 0;
+  for (int o = 0; o < H; ++o) {
+    const float ro = rs[qq * H + o];
+    rank += (ro > r) || (ro == r && o < h);
+  }
+  if (rank < m) {
+    const int64_t dst_row = (int64_t)t * m + rank;
+    heads[dst_row] = h;
+    w_r[dst_row] = __ldg(w + (int64_t)t * H + h);
+    const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)t * H + h) * kD);
+    uint4* dst = reinterpret_cast<uint4*>(q_r + dst_row * kD);
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) dst[i] = __ldg(src + i);
+  }
 }
 
 }  // namespace
@@ -522,8 +567,16 @@ int route_split_count(const misa_problem_t& p, int max_groups, int sms) {
   return n < 2 ? 1 : n;
 }
 
+// Per-slot partial sums [max_groups][nsplit + 1][256] fp32, then one
+// completion counter per group.
 size_t route_split_bytes(int max_groups, int nsplit) {
-  return nsplit <= 1 ? 0 : (size_t)max_groups * (nsplit + 1) * kRouteThreads * sizeof(float);
+  return nsplit <= 1 ? 0
+                     : (size_t)max_groups * (nsplit + 1) * kRouteThreads * sizeof(float) +
+                           (size_t)max_groups * sizeof(int);
+}
+
+int* route_split_counters(float* partial, int max_groups, int nsplit) {
+  return reinterpret_cast<int*>(partial + (size_t)max_groups * (nsplit + 1) * kRouteThreads);
 }
 
 int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, const uint16_t* K,
@@ -535,39 +588,31 @@ int launch_route(const misa_problem_t& p, const uint16_t* q, const float* w, con
   const int sms = num_sms();
   int rc;
   if (nsplit <= 1 || !partial) {
-    if ((rc = set_smem_limit((const void*)route_kernel<kWhole>, smem))) return rc;
+    if ((rc = set_smem_limit((const void*)route_kernel, smem))) return rc;
     ProfScope ps("route", st);
-    return cuda_fail(launch_pdl(route_kernel<kWhole>, dim3(max_groups), dim3(kRouteThreads),
-                                smem, st, q, w, K, Kbar, p.key_offsets, p.block_offsets,
-                                p.q_pos, groups, group_count, p.num_heads, p.block, m, G, heads,
-                                q_r, w_r, router_scores, status_ptr(), 1, sms,
-                                (float*)nullptr),
+    return cuda_fail(launch_pdl(route_kernel, dim3(max_groups), dim3(kRouteThreads), smem, st,
+                                q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups,
+                                group_count, p.num_heads, p.block, m, G, heads, q_r, w_r,
+                                router_scores, status_ptr()),
                      "route_kernel");
   }
-  if ((rc = set_smem_limit((const void*)route_kernel<kFinish>, smem))) return rc;
-  {
-    // One CTA per (group, range) and one per group for its partial block:
-    // the device uses the first count * (ns + 1) of the grid, at most
-    // max(sms, 2 * count) since ns + 1 <= max(2, sms / count).
-    ProfScope ps("route", st);
-    const int ranged = (int)std::min<int64_t>((int64_t)max_groups * (nsplit + 1),
-                                              std::max(sms, 2 * max_groups));
-    const int G8 = (G + 7) / 8 * 8;
-    const int msmem = (2 * kChunk * kRowW + 2 * G8 * kRowW) * (int)sizeof(uint32_t) +
-                      G * kD * (int)sizeof(float);
-    if ((rc = set_smem_limit((const void*)route_mma_kernel, msmem))) return rc;
-    rc = cuda_fail(launch_pdl(route_mma_kernel, dim3(ranged), dim3(kMmaBlock), msmem, st, q, K,
+  // One CTA per (group, range) and one per group for its partial blocks: the
+  // device uses the first count * (ns + 1) of the grid, at most
+  // max(sms, 2 * count) since ns + 1 <= max(2, sms / count).  The last CTA
+  // of each group to finish ranks its heads.
+  ProfScope ps("route", st);
+  const int ranged = (int)std::min<int64_t>((int64_t)max_groups * (nsplit + 1),
+                                            std::max(sms, 2 * max_groups));
+  const int G8 = (G + 7) / 8 * 8;
+  const int msmem = (2 * kChunk * kRowW + 2 * G8 * kRowW) * (int)sizeof(uint32_t) +
+                    G * kD * (int)sizeof(float) + kRouteThreads * (int)sizeof(float);
+  if ((rc = set_smem_limit((const void*)route_mma_kernel, msmem))) return rc;
+  return cuda_fail(launch_pdl(route_mma_kernel, dim3(ranged), dim3(kMmaBlock), msmem, st, q, K,
                               Kbar, p.key_offsets, p.block_offsets, p.q_pos, groups,
-                              group_count, p.num_heads, p.block, G, nsplit, sms, partial),
-                   "route_mma_kernel (ranges)");
-    if (rc) return rc;
-  }
-  ProfScope ps("route_finish", st);
-  return cuda_fail(launch_pdl(route_kernel<kFinish>, dim3(max_groups), dim3(kRouteThreads),
-                              smem, st, q, w, K, Kbar, p.key_offsets, p.block_offsets, p.q_pos,
-                              groups, group_count, p.num_heads, p.block, m, G, heads, q_r, w_r,
-                              router_scores, status_ptr(), nsplit, sms, partial),
-                   "route_kernel (finish)");
+                              group_count, p.num_heads, p.block, G, nsplit, sms, partial,
+                              route_split_counters(partial, max_groups, nsplit), w, m, heads,
+                              q_r, w_r, router_scores, status_ptr()),
+                   "route_mma_kernel");
 }
 
 }  // namespace misa
