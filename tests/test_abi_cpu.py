@@ -90,3 +90,21 @@ def test_host_argument_errors_without_gpu(misa):
     assert lib.misa_pool_keys_from(rp, 16, None, 16, None) == 1
     # the static-scratch router validates like misa_route and refuses m > H
     assert lib.misa_route_static(rp, 16, 16, 16, 16, 65, 16, 16, 16, None, None) == 1
+
+
+def test_workspace_size_covers_the_selection_after_the_scoring_pass(misa):
+    # 128K prefill, m = 8, k = 2048: candidate lists per query row (62 rows of
+    # 128 lanes x 8 B) for the exact selection after the pass, plus the
+    # double-buffered per-CTA lists and the rest (well under 4 GB more).
+    T = 131072
+    p = _problem(misa, num_queries=T, num_heads=32, block=128, max_seq_len=T, total_keys=T,
+                 total_blocks=T // 128)
+    n = misa.lib.misa_workspace_size(ctypes.byref(p), 8, 2048, 0)
+    lists = T * 62 * 128 * 8
+    assert lists <= n < lists + (4 << 30)
+    # a larger k needs longer lists
+    assert misa.lib.misa_workspace_size(ctypes.byref(p), 8, 8192, 0) > n
+    # a decode batch does not stream: no per-query lists
+    d = _problem(misa, num_seqs=16, num_queries=48, max_seq_len=32768, total_keys=16 * 32768,
+                 total_blocks=16 * 512)
+    assert misa.lib.misa_workspace_size(ctypes.byref(d), 8, 2048, 0) < 64 << 20
