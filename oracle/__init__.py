@@ -21,6 +21,13 @@ What it computes, in the order the method runs, from
                     "Probleemstelling")
   7. recall_iou     token recovery vs DSA, measured as IoU
                     (summary, "Experimentele Resultaten", Token Recovery)
+  8. block_pruned_query  head axis x token axis: after routing, the routed
+                    heads score the pooled blocks, only the best blocks'
+                    tokens are scored (thelatestinai.com papers page, HISA
+                    abstract: block-level coarse filter on pooled blocks,
+                    then the indexer inside the kept blocks; gist.science
+                    summary, "Probleemstelling" and "Betekenis en Claims":
+                    head-axis routing combines with token-axis schemes)
 
 Precision: inputs are the same bytes the GPU sees (bf16 bit patterns widened
 exactly, fp32 head weights widened exactly); every dot product, sum and mean
@@ -42,6 +49,11 @@ Readings the pages leave open (each restated where it is used):
   * Ties: heads by (r desc, head asc); tokens by (I desc, index asc);
     -0 counts as +0.  A prefix shorter than k selects every token and pads
     with index -1 / value -inf.
+  * Block pruning (8.): the block score is the routed heads' indexer score
+    of the pooled key, over the full blocks the query sees; the nb best
+    blocks by (score desc, block asc) are kept, and the query's own
+    incomplete block (keys floor((t+1)/B)*B .. t), when there is one, is
+    always kept.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 (closed forms, hand-worked examples, brute force on tiny inputs, identities
@@ -56,7 +68,8 @@ import numpy as np
 __all__ = [
     "widen_bf16", "pool_keys", "block_offsets", "partial_block_mean", "router_scores",
     "route", "token_scores", "topk", "misa_query", "misa_index", "dense_query",
-    "dense_index", "hier_rerank_query", "hier_index", "recall_iou",
+    "dense_index", "hier_rerank_query", "hier_index", "recall_iou", "block_scores",
+    "block_pruned_query", "block_index",
 ]
 
 
@@ -285,3 +298,67 @@ def recall_iou(A, D) -> tuple[float, float]:
     inter = len(a & d)
     recall = inter / len(d) if d else 1.0
     return recall, inter / len(a | d)
+
+
+def block_scores(q_sel: np.ndarray, w_sel: np.ndarray, Kbar_seq: np.ndarray, t: int,
+                 B: int) -> np.ndarray:
+    """Coarse stage of block pruning: the indexer score of every full pooled
+    block query t can see, with a set of heads,
+        S[b] = sum_j w_sel[j] * ReLU(q_sel[j] . Kbar[b]),  b < floor((t+1)/B)
+    (thelatestinai.com papers page, HISA abstract: pooled block
+    representations are scored to drop irrelevant regions).  The full
+    blocks' values are the pooled table's fp32 rows.
+
+    q_sel: fp64 [h, d]; w_sel: fp64 [h]; Kbar_seq: fp32 [M, d] -> fp64 [full].
+    """
+    full = (t + 1) // B
+    dots = q_sel @ Kbar_seq[:full].astype(np.float64).T          # [h, full]
+    return w_sel @ np.maximum(dots, 0.0)
+
+
+def block_pruned_query(q_t, w_t, K_seq, Kbar_seq, t, B, m, nb, k, heads=None, blocks=None):
+    """One query through routed heads x block pruning.
+
+    1. route (as misa_query), keep m heads;
+    2. block_scores with the routed heads, keep the nb best full blocks by
+       (score desc, block asc) -- `blocks` overrides that choice (the parity
+       harness re-scores with another implementation's block set);
+    3. candidates = the tokens of the kept blocks plus the query's own
+       incomplete block (keys floor((t+1)/B)*B .. t);
+    4. the routed heads score the candidates, top-k by (score desc, token
+       asc) (thelatestinai.com papers page, HISA abstract: token-level
+       refinement inside the kept blocks).
+    Returns dict(r, heads, S, blocks, cand, idx, val).
+    """
+    r = router_scores(q_t, w_t, K_seq, Kbar_seq, t, B)
+    if heads is None:
+        heads = route(r, m)
+    heads = np.asarray(heads, dtype=np.int64)
+    S = block_scores(q_t[heads], w_t[heads], Kbar_seq, t, B)
+    if blocks is None:
+        blocks, _ = topk(S, nb)
+    blocks = np.asarray(blocks, dtype=np.int64)
+    full = (t + 1) // B
+    kept = [int(b) for b in blocks if b >= 0]
+    cand = [b * B + j for b in kept for j in range(B)]
+    cand += list(range(full * B, t + 1))
+    cand = np.array(sorted(cand), dtype=np.int64)
+    fine = hier_rerank_query(q_t[heads], w_t[heads], K_seq, cand, k)
+    return dict(r=r, heads=heads.astype(np.int32), S=S, blocks=blocks.astype(np.int32),
+                cand=cand, idx=fine["idx"], val=fine["val"])
+
+
+def block_index(wl, nb, rows=None, m=None, k=None):
+    """Routed heads x block pruning over the listed query rows of a
+    misa_synth.Workload, nb kept full blocks per query."""
+    m = wl.m if m is None else m
+    k = wl.k if k is None else k
+    Kf = widen_bf16(wl.K_bits)
+    Kbar = pool_keys(Kf, wl.key_offsets, wl.B)
+    out = []
+    for i in _rows(wl, rows):
+        s = int(wl.q_seq[i])
+        K_seq, Kbar_seq = _seq_arrays(wl, Kf, Kbar, s)
+        out.append(block_pruned_query(widen_bf16(wl.q_bits[i]), wl.w[i].astype(np.float64),
+                                      K_seq, Kbar_seq, int(wl.q_pos[i]), wl.B, m, nb, k))
+    return out

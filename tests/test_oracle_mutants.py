@@ -16,6 +16,10 @@ def _pins_fail(monkeypatch, name, fn) -> bool:
               pins.test_single_block_router_is_dsa_of_mean_key, pins.test_selection_invariants]
     checks += [lambda c=c: pins.test_golden_case(c) for c in range(6)]
     checks += [lambda s=s: pins.test_brute_force_tiny(s) for s in range(3)]
+    checks += [lambda c=c: pins.test_block_golden_case(c) for c in range(4)]
+    checks += [lambda s=s: pins.test_block_brute_force_tiny(s) for s in range(4)]
+    checks += [pins.test_block_pruning_keeping_every_block_is_routed_topk,
+               pins.test_block_pruning_with_one_key_blocks_is_routed_topk]
     for chk in checks:
         try:
             chk()
@@ -29,6 +33,8 @@ _orig_router = oracle.router_scores
 _orig_scores = oracle.token_scores
 _orig_topk = oracle.topk
 _orig_partial = oracle.partial_block_mean
+_orig_block_scores = oracle.block_scores
+_orig_block_query = oracle.block_pruned_query
 
 
 def _pool_divide_by_B(K, key_offsets, B):
@@ -94,6 +100,40 @@ def _topk_ascending(I, k):
     return idx, np.where(idx >= 0, -val, val)
 
 
+def _block_scores_no_relu(q_sel, w_sel, Kbar_seq, t, B):
+    full = (t + 1) // B
+    return w_sel @ (q_sel @ Kbar_seq[:full].astype(np.float64).T)
+
+
+def _block_scores_unsigned_w(q_sel, w_sel, Kbar_seq, t, B):
+    return _orig_block_scores(q_sel, np.abs(w_sel), Kbar_seq, t, B)
+
+
+def _block_scores_leak(q_sel, w_sel, Kbar_seq, t, B):
+    # scores the pooled row of the query's own block too (it holds future keys)
+    full = min(len(Kbar_seq), (t + B) // B)
+    dots = q_sel @ Kbar_seq[:full].astype(np.float64).T
+    return w_sel @ np.maximum(dots, 0.0)
+
+
+def _block_query_drops_own_block(q_t, w_t, K_seq, Kbar_seq, t, B, m, nb, k, heads=None,
+                                 blocks=None):
+    res = _orig_block_query(q_t, w_t, K_seq, Kbar_seq, t, B, m, nb, k, heads, blocks)
+    full = (t + 1) // B
+    cand = res["cand"][res["cand"] < full * B]
+    fine = oracle.hier_rerank_query(q_t[res["heads"]], w_t[res["heads"]], K_seq, cand, k)
+    return res | dict(cand=cand, idx=fine["idx"], val=fine["val"])
+
+
+def _block_query_keeps_worst(q_t, w_t, K_seq, Kbar_seq, t, B, m, nb, k, heads=None,
+                             blocks=None):
+    r = oracle.router_scores(q_t, w_t, K_seq, Kbar_seq, t, B)
+    hs = oracle.route(r, m) if heads is None else heads
+    S = oracle.block_scores(q_t[hs], w_t[hs], Kbar_seq, t, B)
+    worst, _ = _orig_topk(-S, nb)
+    return _orig_block_query(q_t, w_t, K_seq, Kbar_seq, t, B, m, nb, k, hs, worst)
+
+
 MUTANTS = [
     ("pool_keys", _pool_divide_by_B),
     ("router_scores", _router_unsigned_w),
@@ -104,6 +144,11 @@ MUTANTS = [
     ("token_scores", _scores_relu_after_weight),
     ("topk", _topk_ties_to_higher_index),
     ("topk", _topk_ascending),
+    ("block_scores", _block_scores_no_relu),
+    ("block_scores", _block_scores_unsigned_w),
+    ("block_scores", _block_scores_leak),
+    ("block_pruned_query", _block_query_drops_own_block),
+    ("block_pruned_query", _block_query_keeps_worst),
 ]
 
 

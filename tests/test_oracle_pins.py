@@ -308,3 +308,98 @@ def test_generator_deterministic_and_shaped():
                           needles=False)
     moved = np.any(plain.K_bits != a.K_bits, axis=1)
     assert moved.sum() == 3 + 2
+
+
+# ---------------------------------------------------------------- block pruning (head axis x token axis)
+BLOCK_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "block_pruned_tiny.json")
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_block_golden_case(case):
+    with open(BLOCK_GOLDEN) as f:
+        g = json.load(f)
+    c = g["cases"][case]
+    K = oracle.widen_bf16(f32_to_bf16_bits(np.array(g["K"], dtype=np.float32)))
+    Kbar = oracle.pool_keys(K, np.array([0, len(K)]), g["B"])
+    np.testing.assert_array_equal(Kbar, np.array(g["Kbar"], dtype=np.float32))
+    q = oracle.widen_bf16(f32_to_bf16_bits(np.array(c["q"], dtype=np.float32)))
+    w = np.array(c["w"], dtype=np.float64)
+    res = oracle.block_pruned_query(q, w, K, Kbar, c["t"], g["B"], c["m"], c["nb"], c["k"])
+    assert res["heads"].tolist() == c["heads"]
+    np.testing.assert_array_equal(res["S"], np.array(c["S"], dtype=np.float64))
+    assert res["blocks"].tolist() == c["blocks"]
+    assert res["cand"].tolist() == c["cand"]
+    assert res["idx"].tolist() == c["idx"]
+    np.testing.assert_array_equal(res["val"], np.array(c["val"], dtype=np.float64))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_block_brute_force_tiny(seed):
+    """Plain loops: block scores of the routed heads on the pooled keys, the
+    nb best full blocks plus the incomplete block, token top-k inside."""
+    rng = np.random.default_rng(300 + seed)
+    H = int(rng.integers(1, 7))
+    B = int(rng.choice([2, 4, 8]))
+    L = int(rng.integers(1, 40))
+    d = int(rng.choice([3, 8]))
+    m = int(rng.integers(1, H + 1))
+    nb = int(rng.integers(1, 4))
+    k = int(rng.integers(1, 12))
+    K = oracle.widen_bf16(f32_to_bf16_bits(rng.standard_normal((L, d)).astype(np.float32)))
+    Kbar = oracle.pool_keys(K, np.array([0, L]), B)
+    Kl = K.tolist()
+    for t in range(L):
+        q = oracle.widen_bf16(f32_to_bf16_bits(rng.standard_normal((H, d)).astype(np.float32)))
+        w = rng.standard_normal(H).astype(np.float32).astype(np.float64)
+        res = oracle.block_pruned_query(q, w, K, Kbar, t, B, m, nb, k)
+        r_ref = _brute_router(q.tolist(), w.tolist(), Kl, t, B)
+        heads = sorted(range(H), key=lambda h: (-r_ref[h], h))[:m]
+        assert res["heads"].tolist() == heads
+        full = (t + 1) // B
+        S = []
+        for b in range(full):
+            mean = [float(np.float32(sum(Kl[s][j] for s in range(b * B, b * B + B)) / B))
+                    for j in range(d)]
+            acc = 0.0
+            for h in heads:
+                dot = sum(q[h][j] * mean[j] for j in range(d))
+                acc += w[h] * (dot if dot > 0 else 0.0)
+            S.append(acc)
+        np.testing.assert_allclose(res["S"], S, rtol=1e-12, atol=1e-15)
+        kept = sorted(range(full), key=lambda b: (-(S[b] + 0.0), b))[:nb]
+        assert res["blocks"].tolist() == kept + [-1] * (nb - len(kept))
+        cand = sorted([b * B + j for b in kept for j in range(B)] + list(range(full * B, t + 1)))
+        assert res["cand"].tolist() == cand
+        I_all = _brute_scores(q.tolist(), w.tolist(), heads, Kl, t)
+        order = sorted(cand, key=lambda s: (-(I_all[s] + 0.0), s))[:k]
+        assert res["idx"].tolist() == order + [-1] * (k - len(order))
+        np.testing.assert_allclose(res["val"][:len(order)], [I_all[s] for s in order],
+                                   rtol=1e-12, atol=1e-15)
+
+
+def test_block_pruning_keeping_every_block_is_routed_topk():
+    """Identity: with every full block kept the candidates are the whole
+    prefix, so the result is MISA's routed top-k."""
+    wl = _small_wl()
+    L = int(np.max(wl.seq_lens))
+    pruned = oracle.block_index(wl, nb=L)
+    misa = oracle.misa_index(wl)["rows"]
+    for a, b in zip(pruned, misa):
+        np.testing.assert_array_equal(a["heads"], b["heads"])
+        np.testing.assert_array_equal(a["idx"], b["idx"])
+        np.testing.assert_allclose(a["val"], b["val"], rtol=1e-13)
+
+
+def test_block_pruning_with_one_key_blocks_is_routed_topk():
+    """Special case B = 1: a pooled block is its key (bf16 -> fp32 exact), the
+    block score is the token score, so keeping the k best blocks keeps MISA's
+    routed top-k tokens."""
+    wl = make_workload(seq_lens=[45, 70], queries=[[0, 7, 8, 30, 44], [3, 15, 16, 69]],
+                       H=8, d=16, B=1, m=3, k=10, seed=9, k_cand=25)
+    pruned = oracle.block_index(wl, nb=wl.k)
+    misa = oracle.misa_index(wl)["rows"]
+    for a, b in zip(pruned, misa):
+        np.testing.assert_array_equal(a["idx"], b["idx"])
+        np.testing.assert_allclose(a["val"], b["val"], rtol=1e-13)
+        assert sorted(x for x in a["blocks"].tolist() if x >= 0) == \
+            sorted(x for x in b["idx"].tolist() if x >= 0)
