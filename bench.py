@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-blocks", action="store_true",
+                    help="skip the routed-heads x block-pruning comparison (decode workloads)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--max-queries", type=int, default=0,
                     help="keep only the last N queries (small captures for ncu)")
@@ -536,6 +538,7 @@ def run_ours(args):
             "gpu_launches": gpu_launches, "clocks": clk}
     if decode:
         line["config"]["decode_step"] = "pooled keys of earlier blocks kept; blocks with new keys re-pooled"
+    misa_idx = ix.idx.clone()  # this step's selection, before the comparisons overwrite it
 
     # ---- dense DSA indexer on the same inputs (the in-run comparison)
     if not args.no_dense:
@@ -575,6 +578,62 @@ def run_ours(args):
                              "unit": UNIT, "misa_speedup": dms / ms_step,
                              "score_kernel_tflops": d_flops / (d_k_ms / 1e3) / 1e12,
                              "score_kernel_frac": d_flops / (d_k_ms / 1e3) / 1e12 / peaks["bf16_sustained"]}
+
+    # ---- routed heads x block pruning on the same decode step: the routed
+    # heads score the pooled blocks, only the best 2k/B blocks' tokens (and
+    # the incomplete block) are scored; the step replayed as one CUDA graph.
+    if decode and not args.no_blocks:
+        nb = max(1, 2 * wl.k // wl.B)
+        bx = misa.Indexer(prob, m=wl.m, k=wl.k, n_blocks=nb, device=dev)
+        misa.pool_keys(prob, K, bx.Kbar)
+        blk_run = lambda: bx.blocks(q, w, K, pool_from=pool_from)
+        blk_steps = max(1, min(args.steps, 5))
+        l2_flush()
+        blk_run()
+        torch.cuda.synchronize()
+        bgraph = capture(blk_run) if use_graph else None
+        brun = bgraph.replay if bgraph is not None else blk_run
+        barrier(world)
+        bevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(blk_steps)]
+        for e0, e1 in bevs:
+            settle()
+            e0.record()
+            brun()
+            e1.record()
+        torch.cuda.synchronize()
+        bms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bevs), world) / blk_steps
+        misa.profile_enable(True)
+        for _ in range(blk_steps):
+            settle()
+            blk_run()
+        torch.cuda.synchronize()
+        bprof = misa.profile_collect()
+        misa.profile_enable(False)
+        code, bits = misa.stream_status()
+        if code != 0:
+            raise RuntimeError(f"device status {code} ({bits}) in the block-pruned step")
+
+        def mean_recall(A, D):
+            A, D = A.cpu().numpy(), D.cpu().numpy()
+            rs = []
+            for a, d in zip(A, D):
+                dset = set(int(x) for x in d if x >= 0)
+                if dset:
+                    rs.append(len(dset & set(int(x) for x in a if x >= 0)) / len(dset))
+            return float(np.mean(rs)) if rs else 1.0
+
+        blk = {"n_blocks": nb, "candidates_per_query": (nb + 1) * wl.B,
+               "ms_per_step": bms, "value": job_throughput(pairs, world, bms), "unit": UNIT,
+               "speedup_vs_misa": ms_step / bms,
+               "recall_of_misa_selection": mean_recall(bx.idx, misa_idx),
+               "kernels": {n: {"ms_per_step": t / blk_steps, "launches_per_step": c / blk_steps}
+                           for n, (t, c) in bprof.items()}}
+        if "dense_dsa" in line:
+            blk["speedup_vs_dense"] = line["dense_dsa"]["ms_per_step"] / bms
+            blk["recall_of_dense_selection"] = mean_recall(bx.idx, ix.idx)
+            line["dense_dsa"]["recall_of_dense_selection_by_misa"] = mean_recall(misa_idx, ix.idx)
+        line["block_pruned"] = blk
 
     # ---- end to end through the public API with host buffers.  Every step
     # copies its inputs from pinned host memory and reads its results back;

@@ -179,6 +179,36 @@ int misa_hier_rerank(const misa_problem_t* p, const uint16_t* q, const float* w,
                      const uint16_t* K, const int32_t* cand, int32_t k_cand, int32_t k,
                      int32_t* idx, float* val, void* ws, size_t ws_bytes, misa_stream_t stream);
 
+/* Head axis x token axis -- routed heads with block pruning.  The heads the
+ * router kept (q_r, w_r of misa_route) first score the pooled key blocks,
+ *     S[t,b] = sum_{j<m} w_r[t,j] * ReLU(q_r[t,j] . Kbar[b]),
+ * over the full blocks b < floor((q_pos[t]+1)/B) of the query's sequence;
+ * the n_blocks best blocks by (S desc, block asc) are kept (HISA abstract on
+ * the thelatestinai.com papers page: a block-level coarse filter on pooled
+ * block representations, then token-level refinement inside the kept
+ * blocks; gist.science summary of the MISA paper, "Betekenis en Claims":
+ * head-axis routing combines with token-level schemes).  The candidates are
+ * the keys of the kept blocks plus the keys floor((q_pos[t]+1)/B)*B ..
+ * q_pos[t] of the query's own incomplete block; the routed heads score them
+ * (as misa_score_topk does the whole prefix) and the top-k is kept.  A query
+ * with fewer than n_blocks full blocks keeps them all, so with n_blocks >=
+ * ceil(max_seq_len / B) the result is misa_score_topk's.
+ *   q_r [T, m, 128] bf16, w_r [T, m] fp32 (from misa_route); K; Kbar
+ *   (misa_pool_keys); m a power of two <= min(64, H);
+ *   n_blocks >= 1 with (n_blocks + 1) * B <= 65536;
+ *   1 <= k <= (n_blocks + 1) * B;
+ *   idx [T, k] int32, val [T, k] fp32 as in misa_score_topk;
+ *   blocks: NULL, or [T, n_blocks] int32 receiving the kept block indices
+ *   within the sequence (rank order, -1 padding);
+ *   ws: misa_block_workspace_size(p, n_blocks) bytes, 256-byte aligned.
+ * Five launches on `stream` (block scores, block top-k, candidate
+ * expansion, candidate scoring, top-k); no host synchronisation. */
+size_t misa_block_workspace_size(const misa_problem_t* p, int32_t n_blocks);
+int misa_block_score_topk(const misa_problem_t* p, const uint16_t* q_r, const float* w_r,
+                          int32_t m, const uint16_t* K, const float* Kbar, int32_t n_blocks,
+                          int32_t k, int32_t* idx, float* val, int32_t* blocks, void* ws,
+                          size_t ws_bytes, misa_stream_t stream);
+
 /* The dense DSA indexer, the in-run comparison (MISA abstract; gist.science
  * summary, "Probleemstelling"): every head scores every prefix token.
  *     I[t,s] = sum_{h<H} w[t,h] * ReLU(q[t,h] . K[s])

@@ -9,7 +9,9 @@ without a built libmisa.so raises ImportError (build it with
 Method: "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
 Inference" -- a block-pooled router keeps m of the H indexer heads per query,
 only those heads score the causal prefix, and a per-query top-k follows;
-MISA-dagger re-ranks an enlarged candidate set with all H heads.
+MISA-dagger re-ranks an enlarged candidate set with all H heads; block
+pruning lets the routed heads score only the tokens of the best pooled
+blocks.
 """
 from __future__ import annotations
 
@@ -20,6 +22,7 @@ __all__ = [
     "LIB_PATH", "lib", "MisaError", "Problem", "workspace_size", "block_offsets", "pool_keys",
     "route", "pool_keys_from", "score_topk", "hier_rerank", "dsa_index_dense", "stream_status",
     "selftest_timeout", "route_static", "EXPORTED", "Indexer", "profile_enable", "profile_collect",
+    "block_workspace_size", "block_score_topk",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmisa.so")
@@ -30,7 +33,7 @@ EXPORTED = (
     "misa_route",
     "misa_route_static", "misa_score_topk", "misa_hier_rerank", "dsa_index_dense", "misa_stream_status",
     "misa_selftest_timeout", "misa_profile_enable", "misa_profile_collect",
-    "misa_last_error_string",
+    "misa_last_error_string", "misa_block_workspace_size", "misa_block_score_topk",
 )
 
 if not os.path.exists(LIB_PATH):
@@ -73,6 +76,9 @@ _sig = {
     "misa_profile_collect": (ctypes.c_int, [_c_i32, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                             ctypes.POINTER(_c_i64)]),
     "misa_last_error_string": (ctypes.c_char_p, []),
+    "misa_block_workspace_size": (_c_sz, [_PP, _c_i32]),
+    "misa_block_score_topk": (ctypes.c_int, [_PP, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_i32, _c_i32,
+                                             _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(lib, _name)
@@ -214,6 +220,20 @@ def dsa_index_dense(prob: Problem, q, w, K, k: int, idx, val, ws, scores_dbg=Non
            "dsa_index_dense")
 
 
+def block_workspace_size(prob: Problem, n_blocks: int) -> int:
+    n = lib.misa_block_workspace_size(prob.ref, n_blocks)
+    if n == 0:
+        raise MisaError(1, "misa_block_workspace_size")
+    return int(n)
+
+
+def block_score_topk(prob: Problem, q_r, w_r, m: int, K, Kbar, n_blocks: int, k: int, idx, val,
+                     ws, blocks=None, stream=None) -> None:
+    _check(lib.misa_block_score_topk(prob.ref, _ptr(q_r), _ptr(w_r), m, _ptr(K), _ptr(Kbar),
+                                     n_blocks, k, _ptr(idx), _ptr(val), _ptr(blocks), _ptr(ws),
+                                     ws.numel(), _stream(stream)), "misa_block_score_topk")
+
+
 def stream_status(stream=None) -> int:
     """Synchronise the stream; return (code, status bits) and clear the status word."""
     st = _c_i32(0)
@@ -251,12 +271,14 @@ class Indexer:
     misa():   pool_keys -> route -> score_topk            (MISA)
     hier():   pool_keys -> route -> score_topk(k_cand) -> hier_rerank (MISA-dagger)
     dense():  dsa_index_dense                             (the DSA indexer)
+    blocks(): pool_keys -> route -> block_score_topk      (routed heads x block pruning;
+              needs n_blocks at construction)
     All inputs are device tensors: K uint16/bf16 [total_keys, 128],
     q [T, H, 128] bf16 bits, w [T, H] float32.
     """
 
     def __init__(self, prob: Problem, m: int, k: int, k_cand: int = 0, device="cuda",
-                 with_router_scores: bool = False):
+                 with_router_scores: bool = False, n_blocks: int = 0):
         import torch
         self.prob, self.m, self.k, self.k_cand = prob, m, k, k_cand
         T, H = prob.T, prob.H
@@ -274,6 +296,11 @@ class Indexer:
         if k_cand:
             self.cand = torch.empty((T, k_cand), dtype=torch.int32, device=dev)
             self.cand_val = torch.empty((T, k_cand), dtype=torch.float32, device=dev)
+        self.n_blocks = n_blocks
+        if n_blocks:
+            self.block_ws = torch.empty(block_workspace_size(prob, n_blocks), dtype=torch.uint8,
+                                        device=dev)
+            self.blocks_kept = torch.empty((T, n_blocks), dtype=torch.int32, device=dev)
 
     def pool_route(self, q, w, K, stream=None, pool_from=None):
         """pool_from: None re-pools every block; else an int32 device tensor
@@ -297,6 +324,12 @@ class Indexer:
                    self.cand_val, self.ws, None, stream)
         hier_rerank(self.prob, q, w, K, self.cand, self.k_cand, self.k, self.idx, self.val,
                     self.ws, stream)
+        return self.idx, self.val
+
+    def blocks(self, q, w, K, stream=None, pool_from=None):
+        self.pool_route(q, w, K, stream, pool_from)
+        block_score_topk(self.prob, self.q_r, self.w_r, self.m, K, self.Kbar, self.n_blocks,
+                         self.k, self.idx, self.val, self.block_ws, self.blocks_kept, stream)
         return self.idx, self.val
 
     def dense(self, q, w, K, stream=None, scores_dbg=None):

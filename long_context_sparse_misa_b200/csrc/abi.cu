@@ -145,8 +145,7 @@ ProfScope::~ProfScope() {
   if (slot >= 0) cudaEventRecord(t_prof[slot].stop, st);
 }
 
-namespace {
-
+// Argument checks, also used by the block-pruning entry point (blocks.cu).
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int check_problem(const misa_problem_t* p) {
@@ -184,6 +183,8 @@ int check_ptr(const void* ptr, size_t align, const char* name) {
 }
 
 bool pow2_le64(int x) { return x >= 1 && x <= 64 && (x & (x - 1)) == 0; }
+
+namespace {
 
 int64_t row_ld(const misa_problem_t* p) { return ((int64_t)p->max_seq_len + 3) / 4 * 4; }
 

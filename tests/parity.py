@@ -178,3 +178,62 @@ def check_rerank_rows(wl, rows, cand, idx, val, k=None, rep: Report | None = Non
         check_topk(rep, i, I_c, idx[j], val[j], k, tokens=c)
         rep.rows += 1
     return rep
+
+
+def check_block_set(rep: Report, i, S_oracle, blocks_gpu, nb):
+    """Kept pooled blocks (routed heads x block pruning): a set compare with the
+    same near-threshold allowance as the token top-k.  Returns True when the
+    GPU's set is acceptable."""
+    full = len(S_oracle)
+    want = min(nb, full)
+    g = [int(b) for b in blocks_gpu if b >= 0]
+    if len(g) != want or len(set(g)) != want or any(b >= full for b in g):
+        rep.fail(f"row {i}: kept blocks {sorted(g)} invalid ({want} of {full} expected)")
+        return False
+    if sum(1 for b in blocks_gpu if b < 0) != nb - want:
+        rep.fail(f"row {i}: bad block padding")
+        return False
+    ref, _ = oracle.topk(np.asarray(S_oracle, dtype=np.float64), nb)
+    o = set(int(b) for b in ref if b >= 0)
+    if set(g) != o:
+        thr = S_oracle[int(ref[want - 1])]
+        for b in set(g) ^ o:
+            if abs(S_oracle[b] - thr) > tol(thr):
+                rep.fail(f"row {i}: block {b} S={S_oracle[b]:.7g} far from nb-th {thr:.7g}")
+                return False
+        rep.topk_swaps += len(set(g) - o)
+    return True
+
+
+def check_block_rows(wl, rows, heads, blocks, idx, val, nb, k=None, m=None,
+                     rep: Report | None = None):
+    """Routed heads x block pruning: heads against the oracle router, kept
+    blocks against the oracle's block scores with the GPU's heads, then the
+    top-k against the oracle's scores of the candidates the GPU's blocks give."""
+    rep = rep or Report()
+    k = wl.k if k is None else k
+    m = wl.m if m is None else m
+    Kf = oracle.widen_bf16(wl.K_bits)
+    Kbar_o = oracle.pool_keys(Kf, wl.key_offsets, wl.B)
+    boff = oracle.block_offsets(wl.key_offsets, wl.B)
+    for j, i in enumerate(rows):
+        s = int(wl.q_seq[i])
+        t = int(wl.q_pos[i])
+        K_seq = Kf[int(wl.key_offsets[s]):int(wl.key_offsets[s + 1])]
+        Kbar_seq = Kbar_o[boff[s]:boff[s + 1]]
+        q_t = oracle.widen_bf16(wl.q_bits[i])
+        w_t = wl.w[i].astype(np.float64)
+        r_o = oracle.router_scores(q_t, w_t, K_seq, Kbar_seq, t, wl.B)
+        if not check_heads(rep, i, r_o, heads[j], m):
+            continue
+        use = np.asarray(heads[j], dtype=np.int64)
+        S_o = oracle.block_scores(q_t[use], w_t[use], Kbar_seq, t, wl.B)
+        if not check_block_set(rep, i, S_o, blocks[j], nb):
+            continue
+        res = oracle.block_pruned_query(q_t, w_t, K_seq, Kbar_seq, t, wl.B, m, nb, k,
+                                        heads=use, blocks=blocks[j])
+        c = res["cand"]
+        I_c = oracle.token_scores(q_t[use], w_t[use], K_seq[c])
+        check_topk(rep, i, I_c, idx[j], val[j], k, tokens=c)
+        rep.rows += 1
+    return rep

@@ -108,3 +108,26 @@ def test_workspace_size_covers_the_selection_after_the_scoring_pass(misa):
     d = _problem(misa, num_seqs=16, num_queries=48, max_seq_len=32768, total_keys=16 * 32768,
                  total_blocks=16 * 512)
     assert misa.lib.misa_workspace_size(ctypes.byref(d), 8, 2048, 0) < 64 << 20
+
+
+def test_block_pruning_arguments_and_workspace_without_gpu(misa):
+    lib = misa.lib
+    # decode batch 16 x 32K, B = 64, 64 kept blocks: score rows of 512 pooled
+    # blocks, 65 x 64 candidates per query
+    d = _problem(misa, num_seqs=16, num_queries=48, max_seq_len=32768, total_keys=16 * 32768,
+                 total_blocks=16 * 512)
+    rp = ctypes.byref(d)
+    n = lib.misa_block_workspace_size(rp, 64)
+    per_query = 2 * 512 * 4 + 2 * 64 * 4 + 2 * 65 * 64 * 4
+    assert 48 * per_query <= n < 48 * per_query + 6 * 256
+    assert lib.misa_block_workspace_size(rp, 0) == 0                 # n_blocks >= 1
+    assert lib.misa_block_workspace_size(rp, 1024) == 0              # (n+1)*B > 65536
+    assert b"n_blocks" in lib.misa_last_error_string()
+    args = lambda m, nb, k, ws_bytes, q=16: lib.misa_block_score_topk(
+        rp, q, 16, m, 16, 16, nb, k, 16, 16, None, 256, ws_bytes, None)
+    assert args(6, 64, 2048, n) == 2           # m not a power of two
+    assert args(128, 64, 2048, n) == 2         # m > H
+    assert args(8, 64, 0, n) == 1              # k < 1
+    assert args(8, 8, 2048, n) == 1            # k > (n_blocks + 1) * B
+    assert args(8, 64, 2048, n, q=18) == 1     # misaligned q_r
+    assert args(8, 64, 2048, n - 1) == 3       # workspace too small
