@@ -245,6 +245,18 @@ def workload_config(wl, cfg):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
+def mean_recall(A, D) -> float:
+    """Mean over rows of |A ∩ D| / |D| for two [rows, k] index arrays (-1 =
+    padding; rows with an empty D are skipped): how much of selection D the
+    selection A recovers."""
+    rs = []
+    for a, d in zip(A, D):
+        dset = set(int(x) for x in d if x >= 0)
+        if dset:
+            rs.append(len(dset & set(int(x) for x in a if x >= 0)) / len(dset))
+    return sum(rs) / len(rs) if rs else 1.0
+
+
 def cpu_model() -> str:
     try:
         with open("/proc/cpuinfo") as f:
@@ -614,25 +626,19 @@ def run_ours(args):
         if code != 0:
             raise RuntimeError(f"device status {code} ({bits}) in the block-pruned step")
 
-        def mean_recall(A, D):
-            A, D = A.cpu().numpy(), D.cpu().numpy()
-            rs = []
-            for a, d in zip(A, D):
-                dset = set(int(x) for x in d if x >= 0)
-                if dset:
-                    rs.append(len(dset & set(int(x) for x in a if x >= 0)) / len(dset))
-            return float(np.mean(rs)) if rs else 1.0
-
         blk = {"n_blocks": nb, "candidates_per_query": (nb + 1) * wl.B,
                "ms_per_step": bms, "value": job_throughput(pairs, world, bms), "unit": UNIT,
                "speedup_vs_misa": ms_step / bms,
-               "recall_of_misa_selection": mean_recall(bx.idx, misa_idx),
+               "recall_of_misa_selection": mean_recall(bx.idx.cpu().numpy(),
+                                                         misa_idx.cpu().numpy()),
                "kernels": {n: {"ms_per_step": t / blk_steps, "launches_per_step": c / blk_steps}
                            for n, (t, c) in bprof.items()}}
         if "dense_dsa" in line:
             blk["speedup_vs_dense"] = line["dense_dsa"]["ms_per_step"] / bms
-            blk["recall_of_dense_selection"] = mean_recall(bx.idx, ix.idx)
-            line["dense_dsa"]["recall_of_dense_selection_by_misa"] = mean_recall(misa_idx, ix.idx)
+            dense_idx = ix.idx.cpu().numpy()
+            blk["recall_of_dense_selection"] = mean_recall(bx.idx.cpu().numpy(), dense_idx)
+            line["dense_dsa"]["recall_of_dense_selection_by_misa"] = mean_recall(
+                misa_idx.cpu().numpy(), dense_idx)
         line["block_pruned"] = blk
 
     # ---- end to end through the public API with host buffers.  Every step

@@ -93,3 +93,12 @@ def test_cpu_baseline_samples_the_oracle_on_all_cores_and_one_thread():
     assert out["value"] > 0 and out["cores"] >= 1
     assert "value_1core" in out and out["value_1core"] > 0
     assert out["cpu_model"]
+
+
+def test_mean_recall_of_two_selections():
+    import numpy as np
+    A = np.array([[1, 2, 3, -1], [5, 6, 7, 8], [-1, -1, -1, -1]])
+    D = np.array([[3, 2, 9, -1], [8, 7, 6, 5], [-1, -1, -1, -1]])
+    # row 0: {2,3} of {2,3,9}; row 1: all four; row 2 skipped (empty D)
+    assert abs(bench.mean_recall(A, D) - (2 / 3 + 1.0) / 2) < 1e-12
+    assert bench.mean_recall(D[2:], D[2:]) == 1.0
