@@ -403,3 +403,32 @@ def test_block_pruning_with_one_key_blocks_is_routed_topk():
         np.testing.assert_allclose(a["val"], b["val"], rtol=1e-13)
         assert sorted(x for x in a["blocks"].tolist() if x >= 0) == \
             sorted(x for x in b["idx"].tolist() if x >= 0)
+
+
+def test_block_pruning_causality_and_growing_block_budget():
+    """Keys after the query's position change nothing (their pooled block is
+    never scored, the incomplete block stops at the query); and keeping more
+    blocks only adds candidates, so the kept top-k score never drops."""
+    import dataclasses
+    wl = _small_wl()
+    base = oracle.block_index(wl, nb=2)
+    for i in range(wl.T):
+        s = int(wl.q_seq[i])
+        t = int(wl.q_pos[i])
+        k0, k1 = int(wl.key_offsets[s]), int(wl.key_offsets[s + 1])
+        K2 = wl.K_bits.copy()
+        K2[k0 + t + 1:k1] = f32_to_bf16_bits(np.full((k1 - k0 - t - 1, wl.d), 3.0, np.float32))
+        row = oracle.block_index(dataclasses.replace(wl, K_bits=K2), nb=2, rows=[i])[0]
+        np.testing.assert_array_equal(row["S"], base[i]["S"])
+        np.testing.assert_array_equal(row["idx"], base[i]["idx"])
+    prev = None
+    for nb in range(1, 7):
+        rows = oracle.block_index(wl, nb=nb)
+        if prev is not None:
+            for a, b in zip(prev, rows):
+                assert set(a["cand"].tolist()) <= set(b["cand"].tolist())
+                va, vb = a["val"][a["idx"] >= 0], b["val"][b["idx"] >= 0]
+                assert len(vb) >= len(va)
+                if len(va):
+                    assert np.all(np.sort(vb)[::-1][:len(va)] >= np.sort(va)[::-1] - 1e-15)
+        prev = rows
