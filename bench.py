@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-blocks", action="store_true",
                     help="skip the routed-heads x block-pruning comparison (decode workloads)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the --config workload (no per_config object)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--max-queries", type=int, default=0,
                     help="keep only the last N queries (small captures for ncu)")
@@ -245,18 +247,6 @@ def workload_config(wl, cfg):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def mean_recall(A, D) -> float:
-    """Mean over rows of |A ∩ D| / |D| for two [rows, k] index arrays (-1 =
-    padding; rows with an empty D are skipped): how much of selection D the
-    selection A recovers."""
-    rs = []
-    for a, d in zip(A, D):
-        dset = set(int(x) for x in d if x >= 0)
-        if dset:
-            rs.append(len(dset & set(int(x) for x in a if x >= 0)) / len(dset))
-    return sum(rs) / len(rs) if rs else 1.0
-
-
 def cpu_model() -> str:
     try:
         with open("/proc/cpuinfo") as f:
@@ -356,72 +346,136 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
-    import numpy as np
+def recall_iou_rows(A, D):
+    """Token recovery of selection A against the dense selection D, row by
+    row, averaged over the rows where D is not empty: recall |A n D| / |D| and
+    IoU |A n D| / |A u D| (index -1 = padding).  A, D: torch int32 [rows, k]
+    (any device); runs as torch sorts and searches on that device."""
     import torch
+    a = torch.sort(A, dim=1).values
+    d = torch.sort(D, dim=1).values.contiguous()
+    pos = torch.searchsorted(d, a).clamp_(max=d.shape[1] - 1)
+    inter = ((torch.gather(d, 1, pos) == a) & (a >= 0)).sum(1).double()
+    na, nd = (A >= 0).sum(1).double(), (D >= 0).sum(1).double()
+    keep = nd > 0
+    if not bool(keep.any()):
+        return 1.0, 1.0
+    recall = (inter[keep] / nd[keep]).mean().item()
+    iou = (inter[keep] / (na[keep] + nd[keep] - inter[keep])).mean().item()
+    return recall, iou
 
-    import long_context_sparse_misa_b200 as misa
-    from misa_synth import make_config
 
-    world, rank, local = dist_init()
-    cfg = args.config
-    wl = make_config(cfg, seed=rank_seed(cfg, rank))
-    if args.k_cand >= 0:
-        wl = dataclasses.replace(wl, k_cand=args.k_cand)
-    if args.max_queries and args.max_queries < wl.T:
-        wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
-    hier = bool(wl.k_cand)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    prob = misa.Problem.from_workload(wl, device=dev)
-    K = torch.from_numpy(wl.K_bits).to(dev)
-    q = torch.from_numpy(wl.q_bits).to(dev)
-    w = torch.from_numpy(wl.w).to(dev)
-    ix = misa.Indexer(prob, m=wl.m, k=wl.k, k_cand=wl.k_cand, device=dev)
-    from misa_synth import CONFIGS
-    decode = CONFIGS[cfg]["queries"] != "all"
-    use_graph = args.graph == "on" or (args.graph == "auto" and decode)
-    # Decode step: the keys before this step's queries were pooled by earlier
-    # steps, so only the blocks holding the new keys are re-pooled.
-    pool_from = None
-    if decode:
-        q_per_seq = np.diff(wl.query_offsets)
-        pool_from = torch.tensor(wl.seq_lens - q_per_seq, dtype=torch.int32, device=dev)
-        misa.pool_keys(prob, K, ix.Kbar)
-    run = ((lambda: ix.hier(q, w, K, pool_from=pool_from)) if hier
-           else (lambda: ix.misa(q, w, K, pool_from=pool_from)))
-    eager_run = run
-    small_inputs = wl.q_bits.nbytes + wl.K_bits.nbytes < 2 * 126e6
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small_inputs else None
-    # Read after the write: the flush's own dirty lines are written back here,
-    # outside the timed step, and L2 is left holding clean unrelated lines.
-    clean = torch.ones(64 << 20, dtype=torch.int32, device=dev) if small_inputs else None
+def split_prof(prof):
+    """Kernel entries of a misa.profile_collect() record, and its counters
+    (names starting with '#')."""
+    kern = {n: v for n, v in prof.items() if not n.startswith("#")}
+    cnt = {n[1:]: v[1] for n, v in prof.items() if n.startswith("#")}
+    return kern, cnt
 
-    def l2_flush():
-        if flush is not None:
-            flush.fill_(1)
-            clean.sum()
 
-    def step():
-        l2_flush()
-        run()
+def decode_kbytes(wl):
+    """K prefix bytes the decode scorer streams: each group of 256/m queries
+    of a sequence reads its longest prefix once (256 B per key)."""
+    G = 256 // wl.m
+    kbytes = 0
+    for s_ in range(len(wl.seq_lens)):
+        pos = wl.q_pos[wl.query_offsets[s_]:wl.query_offsets[s_ + 1]]
+        for g0 in range(0, len(pos), G):
+            kbytes += (int(pos[g0:g0 + G].max()) + 1) * 256
+    return kbytes
 
-    def settle():
+
+def roofline_of(wl, prof_ms, launches_per_step, streamed, peaks, clk, workload):
+    """Roofline of the dominant kernel (routed scoring) from its CUDA-event
+    time per step."""
+    pairs = wl.pairs
+    tpp = traffic_per_pair("score_stream" if streamed else "score", workload)
+    sec = prof_ms / 1e3
+    if streamed:
+        # prefill: a dense contraction, 2*m*d flops per scored pair.  The
+        # timed region is sub-second, so the burst bf16 peak applies.
+        flops = 2.0 * wl.m * wl.d * pairs
+        achieved = flops / sec / 1e12
+        r = {"kernel": "score_stream_kernel (tcgen05 routed scoring, top-k candidates in the epilogue)",
+             "bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
+             "frac": achieved / peaks["bf16"],
+             "peak_source": f"bf16_tflops, burst ({peaks['source']})",
+             "frac_of_sustained": achieved / peaks["bf16_sustained"],
+             "algorithmic_flops_per_launch": flops / max(launches_per_step, 1)}
+    else:
+        # decode: HBM-bound; each query group streams its prefix of K once
+        # (256 B per key) and writes its fp32 score rows (4 B per pair)
+        abytes = decode_kbytes(wl) + 4 * pairs
+        achieved = abytes / sec / 1e9
+        r = {"kernel": "score_kernel (tcgen05 routed scoring, score rows)",
+             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": achieved / peaks["hbm_gbs"], "peak_source": f"hbm_gbs ({peaks['source']})",
+             "algorithmic_bytes_per_launch": abytes / max(launches_per_step, 1)}
+    r |= {"launches_per_step": launches_per_step, "kernel_ms_per_step": prof_ms,
+          "sm_mhz_median": clk.get("sm_mhz"),
+          "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
+    return r
+
+
+class Bench:
+    """One workload on this rank's GPU: inputs resident in HBM, the indexer's
+    buffers, and the timing helpers shared by every leg."""
+
+    def __init__(self, cfg, args, rank, world, dev):
+        import dataclasses as dc
+
+        import numpy as np
+        import torch
+
+        import long_context_sparse_misa_b200 as misa
+        from misa_synth import CONFIGS, make_config
+        self.misa, self.torch, self.np = misa, torch, np
+        self.cfg, self.args, self.world, self.dev = cfg, args, world, dev
+        wl = make_config(cfg, seed=rank_seed(cfg, rank))
+        if args.k_cand >= 0 and cfg == args.config:
+            wl = dc.replace(wl, k_cand=args.k_cand)
+        if args.max_queries and args.max_queries < wl.T:
+            wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
+        self.wl = wl
+        self.hier = bool(wl.k_cand)
+        self.decode = CONFIGS[cfg]["queries"] != "all"
+        self.workload = CONFIGS[cfg]["name"]
+        self.prob = misa.Problem.from_workload(wl, device=dev)
+        self.K = torch.from_numpy(wl.K_bits).to(dev)
+        self.q = torch.from_numpy(wl.q_bits).to(dev)
+        self.w = torch.from_numpy(wl.w).to(dev)
+        self.ix = misa.Indexer(self.prob, m=wl.m, k=wl.k, k_cand=wl.k_cand, device=dev)
+        self.use_graph = args.graph == "on" or (args.graph == "auto" and self.decode)
+        # Decode step: the keys before this step's queries were pooled by
+        # earlier steps, so only the blocks holding the new keys are re-pooled.
+        self.pool_from = None
+        if self.decode:
+            q_per_seq = np.diff(wl.query_offsets)
+            self.pool_from = torch.tensor(wl.seq_lens - q_per_seq, dtype=torch.int32, device=dev)
+            misa.pool_keys(self.prob, self.K, self.ix.Kbar)
+        small = wl.q_bits.nbytes + wl.K_bits.nbytes < 2 * 126e6
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small else None
+        # Read after the write: the flush's own dirty lines are written back
+        # here, outside the timed step, and L2 is left holding clean lines.
+        self.clean = torch.ones(64 << 20, dtype=torch.int32, device=dev) if small else None
+
+    def l2_flush(self):
+        if self.flush is not None:
+            self.flush.fill_(1)
+            self.clean.sum()
+
+    def settle(self):
         """Between timed intervals: the L2 flush (small inputs only), then a
         ~1 ms device sleep so that the host has queued the whole next step
         before the device reaches it; the events then bracket device time,
         not the host's launch latency."""
-        l2_flush()
-        torch.cuda._sleep(2_000_000)
+        self.l2_flush()
+        self.torch.cuda._sleep(2_000_000)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-    code, bits = misa.stream_status()
-    if code != 0:
-        raise RuntimeError(f"device status {code} ({bits}) after warm-up")
-
-    def capture(fn):
+    def capture(self, fn):
         """One step as a CUDA graph (all of the library's launches)."""
-        side = torch.cuda.Stream(device=dev)
+        torch = self.torch
+        side = torch.cuda.Stream(device=self.dev)
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
             fn()
@@ -432,289 +486,286 @@ def run_ours(args):
             fn()
         return g
 
-    graph = capture(eager_run) if use_graph else None
-    if graph is not None:
-        run = graph.replay
-
-    # ---- timed region (device time, CUDA events, max over ranks)
-    props = torch.cuda.get_device_properties(dev)
-    clocks = Clocks(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks.start()
-    misa.profile_enable(graph is None)
-    clocks.begin()
-    # Each step is bracketed by its own events; the L2 flush (small inputs
-    # only) runs between steps, outside the timed intervals.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    step_prof = []  # per step: {kernel: (ms, launches)}
-    for e0, e1 in evs:
-        settle()
-        e0.record()
-        run()
-        e1.record()
-        if graph is None:
-            # waits for this step's events (the next step's own events are
-            # recorded after the L2 flush and the device sleep)
-            step_prof.append(misa.profile_collect())
-    torch.cuda.synchronize()
-    clocks.end()
-    clk = clocks.stop()
-    misa.profile_enable(False)
-    barrier(world)
-    step_ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
-    ms = max_over_ranks(sum(step_ms), world)
-    p50 = max_over_ranks(step_ms[len(step_ms) // 2], world)
-    p90 = max_over_ranks(step_ms[min(len(step_ms) - 1, (9 * len(step_ms)) // 10)], world)
-    if graph is not None:
-        # Per-kernel times come from the same step launched eagerly (a graph
-        # replay has no per-launch events), outside the timed region.
+    def timed(self, eager, steps, warmup=1, clocks=None):
+        """Device time of `steps` steps (CUDA events around each, max over
+        ranks), plus the per-kernel times of the same steps launched eagerly.
+        A CUDA graph replays decode steps; its kernels get no events, so their
+        per-kernel times come from eager steps after the timed region.
+        Returns (per-step ms sorted, per-step {kernel: (ms, launches)}, counters)."""
+        torch, misa = self.torch, self.misa
+        for _ in range(warmup):
+            self.l2_flush()
+            eager()
         torch.cuda.synchronize()
-        misa.profile_enable(True)
-        for _ in range(args.steps):
-            settle()
-            eager_run()
-            step_prof.append(misa.profile_collect())
+        graph = self.capture(eager) if self.use_graph else None
+        run = graph.replay if graph is not None else eager
         torch.cuda.synchronize()
+        barrier(self.world)
+        misa.profile_enable(graph is None)
+        if clocks is not None:
+            clocks.begin()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        step_prof = []
+        for e0, e1 in evs:
+            self.settle()
+            e0.record()
+            run()
+            e1.record()
+            if graph is None:
+                # waits for this step's events (the next step's own events are
+                # recorded after the L2 flush and the device sleep)
+                step_prof.append(misa.profile_collect())
+        torch.cuda.synchronize()
+        if clocks is not None:
+            clocks.end()
         misa.profile_enable(False)
-    prof = {}
-    for sp in step_prof:
-        for n, (t, c) in sp.items():
-            t0, c0 = prof.get(n, (0.0, 0))
-            prof[n] = (t0 + t, c0 + c)
-    code, bits = misa.stream_status()
-    if code != 0:
-        raise RuntimeError(f"device status {code} ({bits}) in the timed region")
-    ms_step = ms / args.steps
-    pairs = wl.pairs
-    value = job_throughput(pairs, world, ms_step)
+        barrier(self.world)
+        step_ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+        if graph is not None:
+            misa.profile_enable(True)
+            for _ in range(steps):
+                self.settle()
+                eager()
+                step_prof.append(misa.profile_collect())
+            torch.cuda.synchronize()
+            misa.profile_enable(False)
+            del graph
+        code, bits = misa.stream_status()
+        if code != 0:
+            raise RuntimeError(f"device status {code} ({bits}) in {self.workload}")
+        kerns, counters = [], {}
+        for sp in step_prof:
+            k_, c_ = split_prof(sp)
+            kerns.append(k_)
+            for n, v in c_.items():
+                counters[n] = counters.get(n, 0) + v
+        return step_ms, kerns, counters
 
-    # ---- roofline of the dominant kernel (routed scoring on tcgen05)
-    peaks = load_peaks()
-    kname = "score"
-    k_ms, k_launch = prof.get(kname, (float("nan"), 0))
-    streamed = "topk" not in prof
-    launches_per_step = k_launch / args.steps
-    tpp = traffic_per_pair("score_stream" if streamed else "score",
-                           workload_config(wl, cfg)["workload"])
-    if streamed:
-        # prefill: a dense contraction, 2*m*d flops per scored pair
-        flops = 2.0 * wl.m * wl.d * pairs * args.steps
-        achieved = flops / (k_ms / 1e3) / 1e12
-        roofline = {"kernel": "score_stream_kernel (tcgen05 routed scoring, top-k in the epilogue)",
-                    "bound": "tensor",
-                    "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_sustained"],
-                    "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
-                    "algorithmic_flops_per_launch": 2.0 * wl.m * wl.d * pairs / max(launches_per_step, 1)}
-    else:
-        # decode: HBM-bound; each query group streams its prefix of K once
-        # (256 B per key) and writes its fp32 score rows (4 B per pair)
-        G = 256 // wl.m
-        kbytes = 0
-        for s_ in range(len(wl.seq_lens)):
-            pos = wl.q_pos[wl.query_offsets[s_]:wl.query_offsets[s_ + 1]]
-            for g0 in range(0, len(pos), G):
-                kbytes += (int(pos[g0:g0 + G].max()) + 1) * 256
-        abytes = kbytes + 4 * pairs
-        achieved = abytes * args.steps / (k_ms / 1e3) / 1e9
-        roofline = {"kernel": "score_kernel (tcgen05 routed scoring, score rows)",
-                    "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"],
-                    "peak_source": f"hbm_gbs ({peaks['source']})",
-                    "algorithmic_bytes_per_launch": abytes / max(launches_per_step, 1)}
-    roofline |= {"launches_per_step": launches_per_step,
-                 "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
+    def misa_step(self):
+        ix = self.ix
+        if self.hier:
+            return ix.hier(self.q, self.w, self.K, pool_from=self.pool_from)
+        return ix.misa(self.q, self.w, self.K, pool_from=self.pool_from)
+
+
+def summarise_kernels(kerns, steps):
     def pct(vals, q):
         vals = sorted(vals)
         return vals[min(len(vals) - 1, (q * len(vals)) // 100)]
 
-    kernels = {}
-    for n, (t, c) in prof.items():
-        per_step = [sp.get(n, (0.0, 0))[0] for sp in step_prof]
-        kernels[n] = {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps,
-                      "share": t / max(sum(v[0] for v in prof.values()), 1e-9),
-                      "p50_ms": pct(per_step, 50), "p90_ms": pct(per_step, 90)}
-    gpu_launches = sum(c for _, c in prof.values())
+    tot = {}
+    for sp in kerns:
+        for n, (t, c) in sp.items():
+            t0, c0 = tot.get(n, (0.0, 0))
+            tot[n] = (t0 + t, c0 + c)
+    all_ms = max(sum(v[0] for v in tot.values()), 1e-9)
+    out = {}
+    for n, (t, c) in tot.items():
+        per_step = [sp.get(n, (0.0, 0))[0] for sp in kerns]
+        out[n] = {"ms_per_step": t / steps, "launches_per_step": c / steps, "share": t / all_ms,
+                  "p50_ms": pct(per_step, 50), "p90_ms": pct(per_step, 90)}
+    return out
 
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+
+def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
+    """Time one workload: the MISA step (the headline's metric), its roofline,
+    the dense DSA indexer on the same inputs with recall / IoU of MISA's
+    selection against it, and (decode workloads) routed heads x block pruning.
+    Returns (result dict, Bench)."""
+    import torch
+    bn = Bench(cfg, args, rank, world, dev)
+    wl, ix = bn.wl, bn.ix
+    peaks = load_peaks()
+    warm = max(args.warmup, 3)
+    step_ms, kerns, counters = bn.timed(bn.misa_step, steps, warmup=warm, clocks=clocks)
+    clk = clocks.stop() if clocks is not None else {}
+    ms = max_over_ranks(sum(step_ms), world) / steps
+    p50 = max_over_ranks(step_ms[len(step_ms) // 2], world)
+    p90 = max_over_ranks(step_ms[min(len(step_ms) - 1, (9 * len(step_ms)) // 10)], world)
+    kernels = summarise_kernels(kerns, steps)
+    k = kernels.get("score", {"ms_per_step": float("nan"), "launches_per_step": 0})
+    streamed = "topk" not in kernels
+    res = {"workload": bn.workload, "ms_per_step": ms, "latency_ms": ms,
+           "value": job_throughput(wl.pairs, world, ms), "unit": UNIT,
+           "step_ms_p50": p50, "step_ms_p90": p90, "cuda_graph": bn.use_graph,
+           "roofline": roofline_of(wl, k["ms_per_step"], k["launches_per_step"], streamed, peaks,
+                                   clk, bn.workload),
+           "kernels": kernels,
+           "gpu_launches": sum(v["launches_per_step"] for v in kernels.values()) * steps,
+           "rescanned_queries_per_step": counters.get("rescan_queries", 0) / steps}
+    if clk:
+        res["clocks"] = clk
+    misa_idx = ix.idx.clone()  # this step's selection, before the comparisons overwrite it
+
+    if not args.no_dense:
+        dsteps = max(1, min(steps, 5))
+        d_ms, d_kerns, d_cnt = bn.timed(lambda: ix.dense(bn.q, bn.w, bn.K), dsteps, warmup=1)
+        dms = max_over_ranks(sum(d_ms), world) / dsteps
+        d_kernels = summarise_kernels(d_kerns, dsteps)
+        d_k_ms = d_kernels.get("score", {"ms_per_step": float("nan")})["ms_per_step"]
+        rec, iou = recall_iou_rows(misa_idx, ix.idx)
+        res["dense_dsa"] = {
+            "ms_per_step": dms, "value": job_throughput(wl.pairs, world, dms), "unit": UNIT,
+            "misa_speedup": dms / ms,
+            "kernels": {n: v["ms_per_step"] for n, v in d_kernels.items()},
+            "rescanned_queries_per_step": d_cnt.get("rescan_queries", 0) / dsteps}
+        if streamed:
+            d_tf = 2.0 * wl.H * wl.d * wl.pairs / (d_k_ms / 1e3) / 1e12
+            res["dense_dsa"] |= {"score_kernel_tflops": d_tf,
+                                 "score_kernel_frac": d_tf / peaks["bf16"]}
+        # row a8: token recovery of MISA's final selection against the dense
+        # indexer's, every query row of the step
+        res["recall_vs_dense"] = rec
+        res["iou_vs_dense"] = iou
+        res["recall_rows"] = wl.T
+        dense_idx = ix.idx.clone()
+    else:
+        dense_idx = None
+
+    # routed heads x block pruning on the same decode step: the routed heads
+    # score the pooled blocks, only the best 2k/B blocks' tokens (and the
+    # incomplete block) are scored
+    if bn.decode and not args.no_blocks:
+        import long_context_sparse_misa_b200 as misa
+        nb = max(1, 2 * wl.k // wl.B)
+        bx = misa.Indexer(bn.prob, m=wl.m, k=wl.k, n_blocks=nb, device=dev)
+        misa.pool_keys(bn.prob, bn.K, bx.Kbar)
+        bsteps = max(1, min(steps, 5))
+        b_ms, b_kerns, _ = bn.timed(lambda: bx.blocks(bn.q, bn.w, bn.K, pool_from=bn.pool_from),
+                                    bsteps, warmup=1)
+        bms = max_over_ranks(sum(b_ms), world) / bsteps
+        blk = {"n_blocks": nb, "candidates_per_query": (nb + 1) * wl.B,
+               "ms_per_step": bms, "value": job_throughput(wl.pairs, world, bms), "unit": UNIT,
+               "speedup_vs_misa": ms / bms,
+               "recall_of_misa_selection": recall_iou_rows(bx.idx, misa_idx)[0],
+               "kernels": {n: v["ms_per_step"] for n, v in summarise_kernels(b_kerns, bsteps).items()}}
+        if dense_idx is not None:
+            blk["speedup_vs_dense"] = res["dense_dsa"]["ms_per_step"] / bms
+            blk["recall_vs_dense"], blk["iou_vs_dense"] = recall_iou_rows(bx.idx, dense_idx)
+        res["block_pruned"] = blk
+    torch.cuda.synchronize()
+    return res, bn
+
+
+def e2e_leg(bn, args, world):
+    """End to end through the public API with host buffers.  Every step copies
+    its inputs from pinned host memory and reads its results back; the copies
+    run on their own stream, double buffered, so step i+1's upload and step
+    i's download overlap step i's compute (as a serving loop would pipeline
+    them)."""
+    import torch
+    wl, ix, dev = bn.wl, bn.ix, bn.dev
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    K_h, q_h, w_h = pin(wl.K_bits), pin(wl.q_bits), pin(wl.w)
+    e2e_steps = max(2, min(args.steps, 6))
+    ins = [(bn.K, bn.q, bn.w),
+           (torch.empty_like(bn.K), torch.empty_like(bn.q), torch.empty_like(bn.w))]
+    stage = [(torch.empty_like(ix.idx), torch.empty_like(ix.val)) for _ in range(2)]
+    outs_h = [(torch.empty(tuple(ix.idx.shape), dtype=torch.int32).pin_memory(),
+               torch.empty(tuple(ix.val.shape), dtype=torch.float32).pin_memory())
+              for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    xfer = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    api = ix.hier if bn.hier else ix.misa
+
+    def h2d(b):
+        with torch.cuda.stream(xfer):
+            Kd, qd, wd = ins[b]
+            Kd.copy_(K_h, non_blocking=True)
+            qd.copy_(q_h, non_blocking=True)
+            wd.copy_(w_h, non_blocking=True)
+            ev_in[b].record(xfer)
+
+    def compute(b):
+        comp.wait_event(ev_in[b])
+        Kd, qd, wd = ins[b]
+        api(qd, wd, Kd, pool_from=bn.pool_from)  # the public API calls, one by one
+        stage[b][0].copy_(ix.idx)
+        stage[b][1].copy_(ix.val)
+        ev_done[b].record(comp)
+
+    def d2h(b):
+        with torch.cuda.stream(xfer):
+            xfer.wait_event(ev_done[b])
+            outs_h[b][0].copy_(stage[b][0], non_blocking=True)
+            outs_h[b][1].copy_(stage[b][1], non_blocking=True)
+
+    def pipeline(nsteps, e0=None, e1=None):
+        if e0 is not None:
+            e0.record(xfer)
+        h2d(0)
+        if nsteps > 1:
+            h2d(1)
+        for i in range(nsteps):
+            compute(i % 2)
+            d2h(i % 2)
+            if i + 2 < nsteps:
+                h2d(i % 2)  # ordered after this buffer's compute and download
+        if e1 is not None:
+            e1.record(xfer)
+
+    pipeline(2)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipeline(e2e_steps, e0, e1)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    return {"value": job_throughput(wl.pairs, world, ems), "unit": UNIT, "ms_per_step": ems,
+            "h2d_bytes_per_step": K_h.nbytes + q_h.nbytes + w_h.nbytes,
+            "d2h_bytes_per_step": outs_h[0][0].nbytes + outs_h[0][1].nbytes,
+            "pipelined": "uploads and downloads on a copy stream, double buffered"}
+
+
+# The other configurations, each timed like the headline (decode steps as
+# CUDA graphs) with its dense comparison; parity tests cover all five.
+PER_CONFIG = (0, 1, 2, 4)
+
+
+def run_ours(args):
+    import gc
+
+    import torch
+
+    world, rank, local = dist_init()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    props = torch.cuda.get_device_properties(dev)
+    clocks = Clocks(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    clocks.start()
+    res, bn = measure_config(args.config, args, world, rank, dev, args.steps, True, clocks)
+    wl = bn.wl
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 q,k with 1% planted needles; "
                     "w ~ N(0,1)/sqrt(H) fp32)",
-            "config": workload_config(wl, cfg) | {"parallelism": f"independent problem per GPU x{world}"},
-            "latency_ms": ms_step, "step_ms_p50": p50, "step_ms_p90": p90,
-            "cuda_graph": graph is not None,
-            "roofline": roofline, "kernels": kernels,
-            "gpu_launches": gpu_launches, "clocks": clk}
-    if decode:
+            "config": workload_config(wl, args.config) | {
+                "parallelism": f"independent problem per GPU x{world}"}}
+    if bn.decode:
         line["config"]["decode_step"] = "pooled keys of earlier blocks kept; blocks with new keys re-pooled"
-    misa_idx = ix.idx.clone()  # this step's selection, before the comparisons overwrite it
-
-    # ---- dense DSA indexer on the same inputs (the in-run comparison)
-    if not args.no_dense:
-        dense_steps = max(1, min(args.steps, 5))
-        for _ in range(1):
-            l2_flush()
-            ix.dense(q, w, K)
-        torch.cuda.synchronize()
-        dense_run = lambda: ix.dense(q, w, K)
-        dgraph = capture(dense_run) if use_graph else None
-        if dgraph is not None:
-            dense_run = dgraph.replay
-        barrier(world)
-        misa.profile_enable(dgraph is None)
-        devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(dense_steps)]
-        for e0, e1 in devs:
-            settle()
-            e0.record()
-            dense_run()
-            e1.record()
-        torch.cuda.synchronize()
-        dprof = misa.profile_collect()
-        misa.profile_enable(False)
-        dms = max_over_ranks(sum(a.elapsed_time(b) for a, b in devs), world) / dense_steps
-        if dgraph is not None:
-            misa.profile_enable(True)
-            for _ in range(dense_steps):
-                settle()
-                ix.dense(q, w, K)
-            torch.cuda.synchronize()
-            dprof = misa.profile_collect()
-            misa.profile_enable(False)
-        d_k_ms = dprof.get("score", (float("nan"), 0))[0] / dense_steps
-        d_flops = 2.0 * wl.H * wl.d * pairs
-        line["dense_dsa"] = {"ms_per_step": dms, "value": job_throughput(pairs, world, dms),
-                             "unit": UNIT, "misa_speedup": dms / ms_step,
-                             "score_kernel_tflops": d_flops / (d_k_ms / 1e3) / 1e12,
-                             "score_kernel_frac": d_flops / (d_k_ms / 1e3) / 1e12 / peaks["bf16_sustained"]}
-
-    # ---- routed heads x block pruning on the same decode step: the routed
-    # heads score the pooled blocks, only the best 2k/B blocks' tokens (and
-    # the incomplete block) are scored; the step replayed as one CUDA graph.
-    if decode and not args.no_blocks:
-        nb = max(1, 2 * wl.k // wl.B)
-        bx = misa.Indexer(prob, m=wl.m, k=wl.k, n_blocks=nb, device=dev)
-        misa.pool_keys(prob, K, bx.Kbar)
-        blk_run = lambda: bx.blocks(q, w, K, pool_from=pool_from)
-        blk_steps = max(1, min(args.steps, 5))
-        l2_flush()
-        blk_run()
-        torch.cuda.synchronize()
-        bgraph = capture(blk_run) if use_graph else None
-        brun = bgraph.replay if bgraph is not None else blk_run
-        barrier(world)
-        bevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(blk_steps)]
-        for e0, e1 in bevs:
-            settle()
-            e0.record()
-            brun()
-            e1.record()
-        torch.cuda.synchronize()
-        bms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bevs), world) / blk_steps
-        misa.profile_enable(True)
-        for _ in range(blk_steps):
-            settle()
-            blk_run()
-        torch.cuda.synchronize()
-        bprof = misa.profile_collect()
-        misa.profile_enable(False)
-        code, bits = misa.stream_status()
-        if code != 0:
-            raise RuntimeError(f"device status {code} ({bits}) in the block-pruned step")
-
-        blk = {"n_blocks": nb, "candidates_per_query": (nb + 1) * wl.B,
-               "ms_per_step": bms, "value": job_throughput(pairs, world, bms), "unit": UNIT,
-               "speedup_vs_misa": ms_step / bms,
-               "recall_of_misa_selection": mean_recall(bx.idx.cpu().numpy(),
-                                                         misa_idx.cpu().numpy()),
-               "kernels": {n: {"ms_per_step": t / blk_steps, "launches_per_step": c / blk_steps}
-                           for n, (t, c) in bprof.items()}}
-        if "dense_dsa" in line:
-            blk["speedup_vs_dense"] = line["dense_dsa"]["ms_per_step"] / bms
-            dense_idx = ix.idx.cpu().numpy()
-            blk["recall_of_dense_selection"] = mean_recall(bx.idx.cpu().numpy(), dense_idx)
-            line["dense_dsa"]["recall_of_dense_selection_by_misa"] = mean_recall(
-                misa_idx.cpu().numpy(), dense_idx)
-        line["block_pruned"] = blk
-
-    # ---- end to end through the public API with host buffers.  Every step
-    # copies its inputs from pinned host memory and reads its results back;
-    # the copies run on their own stream, double buffered, so step i+1's
-    # upload and step i's download overlap step i's compute (as a serving
-    # loop would pipeline them).
+    line |= {k_: v for k_, v in res.items() if k_ not in ("value", "unit", "ms_per_step", "workload")}
     if not args.no_e2e:
-        pin = lambda a: torch.from_numpy(a).pin_memory()
-        K_h, q_h, w_h = pin(wl.K_bits), pin(wl.q_bits), pin(wl.w)
-        e2e_steps = max(2, min(args.steps, 6))
-        ins = [(K, q, w), (torch.empty_like(K), torch.empty_like(q), torch.empty_like(w))]
-        stage = [(torch.empty_like(ix.idx), torch.empty_like(ix.val)) for _ in range(2)]
-        outs_h = [(torch.empty(tuple(ix.idx.shape), dtype=torch.int32).pin_memory(),
-                   torch.empty(tuple(ix.val.shape), dtype=torch.float32).pin_memory())
-                  for _ in range(2)]
-        comp = torch.cuda.current_stream()
-        xfer = torch.cuda.Stream(device=dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        api = ix.hier if hier else ix.misa
-
-        def h2d(b):
-            with torch.cuda.stream(xfer):
-                Kd, qd, wd = ins[b]
-                Kd.copy_(K_h, non_blocking=True)
-                qd.copy_(q_h, non_blocking=True)
-                wd.copy_(w_h, non_blocking=True)
-                ev_in[b].record(xfer)
-
-        def compute(b):
-            comp.wait_event(ev_in[b])
-            Kd, qd, wd = ins[b]
-            api(qd, wd, Kd, pool_from=pool_from)  # the public API calls, one by one
-            stage[b][0].copy_(ix.idx)
-            stage[b][1].copy_(ix.val)
-            ev_done[b].record(comp)
-
-        def d2h(b):
-            with torch.cuda.stream(xfer):
-                xfer.wait_event(ev_done[b])
-                outs_h[b][0].copy_(stage[b][0], non_blocking=True)
-                outs_h[b][1].copy_(stage[b][1], non_blocking=True)
-
-        def pipeline(nsteps, e0=None, e1=None):
-            if e0 is not None:
-                e0.record(xfer)
-            h2d(0)
-            if nsteps > 1:
-                h2d(1)
-            for i in range(nsteps):
-                compute(i % 2)
-                d2h(i % 2)
-                if i + 2 < nsteps:
-                    h2d(i % 2)  # ordered after this buffer's compute and download
-            if e1 is not None:
-                e1.record(xfer)
-
-        pipeline(2)
-        torch.cuda.synchronize()
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        pipeline(e2e_steps, e0, e1)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-        line["e2e"] = {"value": job_throughput(pairs, world, ems), "unit": UNIT,
-                       "ms_per_step": ems,
-                       "h2d_bytes_per_step": K_h.nbytes + q_h.nbytes + w_h.nbytes,
-                       "d2h_bytes_per_step": outs_h[0][0].nbytes + outs_h[0][1].nbytes,
-                       "pipelined": "uploads and downloads on a copy stream, double buffered"}
-
-    # ---- CPU oracle on this host, rank 0 at N=1
+        line["e2e"] = e2e_leg(bn, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(wl, args.cpu_budget_s,
                                                    one_core_s=args.cpu_budget_s / 4)
-
+    del bn
+    gc.collect()
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_config:
+        per = {}
+        for c in PER_CONFIG:
+            if c == args.config:
+                continue
+            r, b = measure_config(c, args, world, rank, dev, min(args.steps, 10), False)
+            per[r.pop("workload")] = r
+            del b
+            gc.collect()
+            torch.cuda.empty_cache()
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

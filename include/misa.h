@@ -199,7 +199,7 @@ int misa_hier_rerank(const misa_problem_t* p, const uint16_t* q, const float* w,
  *   1 <= k <= (n_blocks + 1) * B;
  *   idx [T, k] int32, val [T, k] fp32 as in misa_score_topk;
  *   blocks: NULL, or [T, n_blocks] int32 receiving the kept block indices
- *   within the sequence (rank order, -1 padding);
+ *   within the sequence (row order unspecified, -1 padding);
  *   ws: misa_block_workspace_size(p, n_blocks) bytes, 256-byte aligned.
  * Five launches on `stream` (block scores, block top-k, candidate
  * expansion, candidate scoring, top-k); no host synchronisation. */
@@ -235,6 +235,11 @@ int misa_selftest_timeout(int32_t wait_ms, misa_stream_t stream);
  * kernel name (names: max_kernels x 32 chars), the summed device time in
  * milliseconds and the launch count, then clears the record.  Returns the
  * number of kernel names (at most max_kernels) or a negative MISA_ERR code.
+ * Names starting with '#' are counters, not kernels (time 0, the count in
+ * `launches`): "#rescan_queries" sums, over the streaming top-k calls traced,
+ * the queries whose sampled threshold did not hold and were rescanned.
+ * While tracing, each such call also queues a 4-byte device-to-host copy
+ * into pinned host memory the library keeps for this purpose.
  * No counterpart in the paper. */
 int misa_profile_enable(int32_t on);
 int misa_profile_collect(int32_t max_kernels, char* names, double* total_ms, int64_t* launches);

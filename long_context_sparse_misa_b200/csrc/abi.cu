@@ -112,6 +112,14 @@ struct ProfRecord {
 thread_local bool t_prof_on = false;
 thread_local std::vector<ProfRecord> t_prof;       // recorded, not yet collected
 thread_local std::vector<cudaEvent_t> t_free_events;
+// Device counters copied back while tracing (pinned host slot, event after the copy).
+struct CountRecord {
+  const char* name;
+  int32_t* slot;
+  cudaEvent_t done;
+};
+thread_local std::vector<CountRecord> t_counts;
+thread_local std::vector<int32_t*> t_free_slots;
 
 cudaEvent_t take_event() {
   if (!t_free_events.empty()) {
@@ -143,6 +151,27 @@ ProfScope::ProfScope(const char* name, cudaStream_t s) : slot(-1), st(s) {
 
 ProfScope::~ProfScope() {
   if (slot >= 0) cudaEventRecord(t_prof[slot].stop, st);
+}
+
+void prof_count(const char* name, const int* dev_count, cudaStream_t st) {
+  if (!t_prof_on) return;
+  int32_t* slot = nullptr;
+  if (!t_free_slots.empty()) {
+    slot = t_free_slots.back();
+    t_free_slots.pop_back();
+  } else if (cudaHostAlloc(reinterpret_cast<void**>(&slot), sizeof(int32_t),
+                           cudaHostAllocDefault) != cudaSuccess) {
+    return;
+  }
+  cudaEvent_t done = take_event();
+  if (!done || cudaMemcpyAsync(slot, dev_count, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+                   cudaSuccess) {
+    t_free_slots.push_back(slot);
+    if (done) t_free_events.push_back(done);
+    return;
+  }
+  cudaEventRecord(done, st);
+  t_counts.push_back({name, slot, done});
 }
 
 // Argument checks, also used by the block-pruning entry point (blocks.cu).
@@ -304,7 +333,7 @@ int score_topk_impl(const misa_problem_t* p, const uint16_t* qsel, const float* 
       a.dcand = reinterpret_cast<uint2*>(db);
       const size_t lists = align_up((size_t)T * a.drows * 128 * sizeof(uint2));
       a.dcnt = reinterpret_cast<int*>(db + lists);
-      a.danchor = reinterpret_cast<int*>(db + lists + align_up((size_t)T * 128 * sizeof(int)));
+      a.danchor = reinterpret_cast<int2*>(db + lists + align_up((size_t)T * 128 * sizeof(int)));
     }
     return launch_score_stream(a, st);
   }
@@ -595,6 +624,20 @@ int misa_profile_collect(int32_t max_kernels, char* names, double* total_ms, int
     t_free_events.push_back(r.stop);
   }
   t_prof.clear();
+  for (auto& c : t_counts) {
+    cudaError_t e = cudaEventSynchronize(c.done);
+    if (e != cudaSuccess) return -cuda_fail(e, "misa_profile_collect");
+    auto it = acc.find(c.name);
+    if (it == acc.end()) {
+      order.push_back(c.name);
+      acc[c.name] = {0.0, *c.slot};
+    } else {
+      it->second.second += *c.slot;
+    }
+    t_free_slots.push_back(c.slot);
+    t_free_events.push_back(c.done);
+  }
+  t_counts.clear();
   int n = 0;
   for (auto& name : order) {
     if (n >= max_kernels) break;

@@ -56,6 +56,11 @@ size_t route_path_bytes(const misa_problem_t* p);
 // Whether tracing (misa_profile_enable) is on for the calling host thread.
 bool tracing_enabled();
 
+// Tracing: copies a device int32 counter back after the work queued on `st`
+// so far; misa_profile_collect adds it under `name` (in the launch-count
+// field).  No effect unless tracing is on.
+void prof_count(const char* name, const int* dev_count, cudaStream_t st);
+
 // Tracing: brackets one kernel launch with events on `st` when profiling is on.
 struct ProfScope {
   ProfScope(const char* name, cudaStream_t st);
@@ -160,7 +165,7 @@ struct StreamArgs {
   // one list per query row, stream_deferred_bytes(T, subcap, k) in all.
   uint2* dcand = nullptr;  // [T][drows][128]
   int* dcnt = nullptr;     // [T][128]
-  int* danchor = nullptr;  // [T]
+  int2* danchor = nullptr; // [T] {histogram base, top score bits}
   int drows = 0;           // stream_deferred_rows(k, subcap)
 };
 int launch_score_stream(const StreamArgs& a, cudaStream_t st);

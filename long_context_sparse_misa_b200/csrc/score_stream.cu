@@ -35,11 +35,12 @@
 //     best score.
 //   * main pass over all tiles: a key is appended to query q's candidates
 //     only if I >= tau_q.  Each (query, TMEM lane) has its own list, so no
-//     lane needs a rank from the others: a passing lane stores to row cnt of
-//     its list and counts (a predicated store and an add, no vote).  Lists
-//     hold kRowsCap rows; a fuller list stops storing and sends its query to
-//     the rescan.  A query's 128 lists are stored row by row, so that a row
-//     of all lists is 1 KB contiguous.
+//     lane needs a rank from the others: a passing lane stores at its list's
+//     next-row pointer and advances it (a compare, a predicated store and a
+//     predicated add, no vote).  Every kCheckTiles tiles a list that could
+//     pass its capacity before the next check stops storing and is marked
+//     full, which sends its query to the rescan.  A query's 128 lists are
+//     stored row by row, so that a row of all lists is 1 KB contiguous.
 //   * check and select: every key scoring at least tau_q was appended, so
 //     if at least min(k, n) keys were appended (and no list ran past its
 //     rows) the exact top-k is among them.  A warp then histograms the
@@ -87,17 +88,18 @@ constexpr int kMaxG = 32;                        // queries per group (m >= 8)
 constexpr int kBins = 256;
 constexpr int kHistWords = kBins / 2;            // two 16-bit bin counts per word
 constexpr int kBinShift = 18;                    // 14-bit score key prefix: 1/32 octave
-constexpr int kHeadroom = 224;                   // bins below the first tile's maximum
+constexpr int kHeadroom = 224;                   // distance bins below the tile's spread
 constexpr int kSelBins = 256;
 constexpr int kProbeStride = 24;                 // probe every 24th tile ...
 constexpr int kProbeOff = 12;                    // ... starting at tile 12
 constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
+constexpr int kCheckTiles = 8;                   // list capacity checked every 8 tiles
 
 static_assert(kSelBins >= kBins, "final-select histogram");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
-                           kMaxG * 4 * 5 /*pos,row,tau,maxkey,base*/ +
+                           kMaxG * 4 * 7 /*pos,row,tau,maxkey,minkey,base,top*/ +
                            kMaxG * kHistWords * 4 /*hist*/ + kSelWarps * kSelBins * 4 /*select*/ +
-                           2 * kMaxG * 4 * 3 /*selector copies of pos,row,base*/ +
+                           2 * kMaxG * 4 * 4 /*selector copies of pos,row,base,top*/ +
                            2 * 4 * 3 /*selnq,selnext,seldone*/ +
                            32 * 8 /*barriers*/ + 16;
 
@@ -108,13 +110,16 @@ struct Smem {
   int* pos;
   int* row;
   float* tau;
-  uint32_t* maxkey;
-  int* base;  // histogram anchor per query
+  uint32_t* maxkey;  // first scored tile's maximum and minimum (order keys)
+  uint32_t* minkey;
+  int* base;    // histogram anchor per query (see Anchor)
+  float* top;
   uint32_t* hist;
   uint32_t* sel;   // [kSelWarps][kSelBins]
-  int* mpos;       // [2][kMaxG] the selectors' copies of pos, row, base
+  int* mpos;       // [2][kMaxG] the selectors' copies of pos, row and the anchor
   int* mrow;
   int* mbase;
+  float* mtop;
   int* selnq;          // [2] queries of the group in each candidate buffer
   int* selnext;        // [2] next query to claim for selection
   int* seldone;        // [2] queries selected
@@ -142,13 +147,16 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.row = s.pos + kMaxG;
   s.tau = reinterpret_cast<float*>(s.row + kMaxG);
   s.maxkey = reinterpret_cast<uint32_t*>(s.tau + kMaxG);
-  s.base = reinterpret_cast<int*>(s.maxkey + kMaxG);
-  s.hist = reinterpret_cast<uint32_t*>(s.base + kMaxG);
+  s.minkey = s.maxkey + kMaxG;
+  s.base = reinterpret_cast<int*>(s.minkey + kMaxG);
+  s.top = reinterpret_cast<float*>(s.base + kMaxG);
+  s.hist = reinterpret_cast<uint32_t*>(s.top + kMaxG);
   s.sel = s.hist + kMaxG * kHistWords;
   s.mpos = reinterpret_cast<int*>(s.sel + kSelWarps * kSelBins);
   s.mrow = s.mpos + 2 * kMaxG;
   s.mbase = s.mrow + 2 * kMaxG;
-  s.selnq = s.mbase + 2 * kMaxG;
+  s.mtop = reinterpret_cast<float*>(s.mbase + 2 * kMaxG);
+  s.selnq = reinterpret_cast<int*>(s.mtop + 2 * kMaxG);
   s.selnext = s.selnq + 2;
   s.seldone = s.selnext + 2;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.seldone + 2);
@@ -166,37 +174,88 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-// Histogram anchor of a query: 7 octaves below its first tile's maximum.
-__device__ __forceinline__ int hist_base(uint32_t maxkey) {
-  const int b = static_cast<int>(maxkey >> kBinShift) - kHeadroom;
-  return b < 0 ? 0 : b;
+// Histogram bins of one query (probe and exact selection).  The anchor is
+// the query's first scored tile, with spread = its largest minus its
+// smallest score.  A score v falls in 1/32-octave bins of its distance below
+// the reference top = (largest score) + spread/4, top - v, over distances
+// from spread/128 to 2 * spread (256 bins, higher bin = higher score); bin
+// 255 also takes every score above top or within spread/128 of it, bin 0
+// every score more than 2 * spread below it.  Measuring from the top of the
+// tile's own range (not from zero) keeps fine bins near the k-th best score
+// whatever its sign: with all H heads, a query whose head weights are mostly
+// negative has its k-th best score near or below zero.  The quarter spread
+// above the tile's maximum leaves room for the many prefixes whose k-th best
+// score lies above the first tile's maximum.  Bin numbers grow with v (the
+// subtraction and the order key are both monotonic), so a bin boundary is a
+// valid threshold.
+struct Anchor {
+  float top;
+  int base;  // order-key bin (key >> kBinShift) of distance spread/128
+};
+
+__device__ __forceinline__ Anchor make_anchor(uint32_t maxkey, uint32_t minkey) {
+  Anchor a;
+  if (maxkey == 0u || minkey > maxkey) {  // no valid score in the tile
+    a.top = 0.f;
+    a.base = static_cast<int>(order_key(1e-30f) >> kBinShift) - kHeadroom;
+    return a;
+  }
+  const float hi = key_to_float(maxkey);
+  const float spread = fmaxf(hi - key_to_float(minkey), 1e-30f);
+  a.top = hi + 0.25f * spread;
+  a.base = static_cast<int>(order_key(spread) >> kBinShift) - kHeadroom;
+  return a;
 }
 
-__device__ __forceinline__ int score_bin(uint32_t key, int base) {
-  const int b = static_cast<int>(key >> kBinShift) - base;
-  return b < 0 ? 0 : (b >= kBins ? kBins - 1 : b);
+__device__ __forceinline__ int dist_bin(float v, float top, int base) {
+  const int j = static_cast<int>(order_key(top - v) >> kBinShift) - base;
+  return kBins - 1 - (j < 0 ? 0 : (j >= kBins ? kBins - 1 : j));
+}
+
+// Lowest score of bin b (b > 0): top minus the upper distance edge of the bin.
+__device__ __forceinline__ float bin_floor(int b, float top, int base) {
+  const int j = kBins - 1 - b;
+  return top - key_to_float(static_cast<uint32_t>(base + j + 1) << kBinShift);
 }
 
 // Columns C*16 .. C*16+15 of a warp's 64: the head-weighted ReLU sums in the
 // order of relu_wsum (even heads into a0, odd into a1, then a0 + a1), with
-// a query's running sums carried across chunks when it spans several.
+// a query's running sums carried across chunks when it spans several.  The
+// halved weights come four at a time (one 16-byte shared load).
 template <int MH, int C, int QH>
 __device__ __forceinline__ void chunk_wsum(const float (&v)[16], const float* wcol, float& a0,
                                            float& a1, float (&sc)[QH]) {
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
+  for (int p = 0; p < 4; ++p) {
     constexpr int kBase = C * 16;
-    const int col = kBase + 2 * p;
-    const int j = col % MH;
-    if (j == 0) {
-      a0 = 0.f;
-      a1 = 0.f;
+    const int col = kBase + 4 * p;
+    const float4 w4 = *reinterpret_cast<const float4*>(wcol + col);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c2 = col + 2 * h;
+      if (c2 % MH == 0) {
+        a0 = 0.f;
+        a1 = 0.f;
+      }
+      const float c0 = v[4 * p + 2 * h], c1 = v[4 * p + 2 * h + 1];
+      ffma2(a0, a1, h ? w4.z : w4.x, h ? w4.w : w4.y, c0 + fabsf(c0), c1 + fabsf(c1));
+      if ((c2 + 2) % MH == 0) sc[c2 / MH] = a0 + a1;
     }
-    const float2 wj = *reinterpret_cast<const float2*>(wcol + col);
-    const float c0 = v[2 * p], c1 = v[2 * p + 1];
-    ffma2(a0, a1, wj.x, wj.y, c0 + fabsf(c0), c1 + fabsf(c1));
-    if (j + 2 == MH) sc[col / MH] = a0 + a1;
   }
+}
+
+// Appends {v, key} at *p and advances p by one list row (128 entries) when
+// v >= tau; one compare, one predicated store, one predicated add.  (No
+// memory clobber: nothing in this thread reads the lists back before a
+// barrier, and the barriers are compiler fences.)
+__device__ __forceinline__ void append_if(uint2*& p, float v, float tau, int key) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ge.f32 q, %1, %2;\n\t"
+      "@q st.global.v2.b32 [%0], {%3, %4};\n\t"
+      "@q add.s64 %0, %0, 1024;\n\t}\n"
+      : "+l"(p)
+      : "f"(v), "f"(tau), "r"(__float_as_uint(v)), "r"(key));
 }
 
 // Barrier over the epilogue warps (bounded; warp-uniform result).
@@ -278,7 +337,7 @@ __device__ __forceinline__ void find_crossing16(const uint32_t* words, int nb, u
 // reads 256 contiguous bytes.  Threshold-bin entries are compacted to the
 // front of their own list, which only rewrites entries that the same lane
 // has already read.
-__device__ void final_select(uint2* region, const int* cnt, int base, int k, int32_t* idx,
+__device__ void final_select(uint2* region, const int* cnt, Anchor anc, int k, int32_t* idx,
                              float* val, uint32_t* selh) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
@@ -328,7 +387,7 @@ __device__ void final_select(uint2* region, const int* cnt, int base, int k, int
       for (int u = 0; u < kR; ++u)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          red_add_shared_if(&selh[score_bin(order_key(__uint_as_float(xv[u][i])), base)],
+          red_add_shared_if(&selh[dist_bin(__uint_as_float(xv[u][i]), anc.top, anc.base)],
                             r0 + u < c[i]);
     }
     __syncwarp();
@@ -352,7 +411,7 @@ __device__ void final_select(uint2* region, const int* cnt, int base, int k, int
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint2 e = ev[u][i];
-          const int b = r0 + u < c[i] ? score_bin(order_key(__uint_as_float(e.x)), base) : -1;
+          const int b = r0 + u < c[i] ? dist_bin(__uint_as_float(e.x), anc.top, anc.base) : -1;
           const uint32_t up = __ballot_sync(kAll, b > bstar);
           const int o = out + __popc(up & lt);
           st_global_u32_if(idx + o, e.y, b > bstar && o < k);
@@ -468,7 +527,7 @@ struct Lists {
   int* cnt;      // [grid][2][slots][128], or [T][128]
   int rows_cap;
   int slots;
-  int* anchor;   // [T] deferred selection; nullptr: selected in the kernel
+  int2* anchor;  // [T] {base, top bits}: deferred selection; nullptr: selected in the kernel
   __device__ __forceinline__ uint2* list_t(int64_t t) const {
     return cand + t * rows_cap * 128;
   }
@@ -507,8 +566,8 @@ __device__ void select_query(const Smem& s, const Lists& ls, const Sched& sc, in
     if (lane == 0 && sc.fail_out) sc.fail_out[atomicAdd(sc.fail_count, 1)] = t;
     return;
   }
-  final_select(ls.list(b, qi), qcnt, s.mbase[b * kMaxG + qi], k, idx_out + (int64_t)t * k,
-               val_out + (int64_t)t * k, selh);
+  final_select(ls.list(b, qi), qcnt, Anchor{s.mtop[b * kMaxG + qi], s.mbase[b * kMaxG + qi]}, k,
+               idx_out + (int64_t)t * k, val_out + (int64_t)t * k, selh);
 }
 
 // Claims queries of candidate buffer b and selects them until none is left.
@@ -719,24 +778,29 @@ __global__ void __maxnreg__(96)
         s.row[et] = qb + et;
         s.tau[et] = p >= 0 ? -INFINITY : INFINITY;  // padding / invalid slots never append
         s.maxkey[et] = 0u;
+        s.minkey[et] = 0xFFFFFFFFu;
       }
       for (int i = et; i < G * kHistWords; i += kEpiThreads) s.hist[i] = 0u;
-      // This lane's list of its warp's first query (row-major over the 128
-      // lists of a query) and its append counts, one per query.
-      uint2* mylist = (deferred ? ls.list_t(qb + half * QH)
-                                : ls.list(bsel, 0) + (int64_t)(half * QH) * ls.rows_cap * 128) +
-                      lrow;
-      const uint32_t qstride = 128u * static_cast<uint32_t>(ls.rows_cap);
-      const int rows_cap = ls.rows_cap;
-      int cnt[QH];
+      // This lane's list of each of its warp's queries (row-major over the 128
+      // lists of a query): qlist(qq) is the first row, nxt[qq] the next row
+      // to write.  A list that comes within kCheckTiles rows of its capacity
+      // (checked every kCheckTiles main-pass tiles, so no store can pass the
+      // end) stops appending and is marked full (one row past capacity).
+      uint2* const mylist =
+          (deferred ? ls.list_t(qb + half * QH)
+                    : ls.list(bsel, 0) + (int64_t)(half * QH) * ls.rows_cap * 128) +
+          lrow;
+      const int64_t qstride = 128 * (int64_t)ls.rows_cap;
+      auto qlist = [&](int qq) { return mylist + qq * qstride; };
+      uint2* nxt[QH];
 #pragma unroll
-      for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
+      for (int qq = 0; qq < QH; ++qq) nxt[qq] = qlist(qq);
       if (!(ok = ep_barrier(s, ephase, status))) break;
       int minpos = 0x7fffffff;  // smallest valid position of the group (-1 if any invalid)
       for (int qi = 0; qi < nq; ++qi) minpos = min(minpos, s.pos[qi]);
       float tauR[QH];  // this warp's copy of its queries' thresholds
 #pragma unroll
-      for (int qq = 0; qq < QH; ++qq) tauR[qq] = -INFINITY;
+      for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
 
       for (int step = 0; step < np + ntiles; ++step, ++tb) {
         const bool probing = step < np;
@@ -773,17 +837,26 @@ __global__ void __maxnreg__(96)
         chunk_wsum<MH, 3>(vB, wcol, a0, a1, sc_);
         const int key = tile * kTileKeys + lrow;
         if (step == 0) {
-          // Anchor every query's histogram at the maximum of its first tile.
+          // Anchor every query's histogram on the range of its first tile.
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) {
             const int qi = half * QH + qq;
-            uint32_t kk = key <= s.pos[qi] ? order_key(sc_[qq]) : 0u;
-            kk = __reduce_max_sync(0xffffffffu, kk);
-            if (lane == 0) atomicMax(&s.maxkey[qi], kk);
+            const bool v = key <= s.pos[qi];
+            const uint32_t kk = order_key(sc_[qq]);
+            const uint32_t hi = __reduce_max_sync(0xffffffffu, v ? kk : 0u);
+            const uint32_t lo = __reduce_min_sync(0xffffffffu, v ? kk : 0xFFFFFFFFu);
+            if (lane == 0) {
+              atomicMax(&s.maxkey[qi], hi);
+              atomicMin(&s.minkey[qi], lo);
+            }
           }
           if (!(ok = ep_barrier(s, ephase, status))) break;
           // every warp of a half writes the same anchors for its queries
-          if (lane < QH) s.base[half * QH + lane] = hist_base(s.maxkey[half * QH + lane]);
+          if (lane < QH) {
+            const Anchor a = make_anchor(s.maxkey[half * QH + lane], s.minkey[half * QH + lane]);
+            s.base[half * QH + lane] = a.base;
+            s.top[half * QH + lane] = a.top;
+          }
           __syncwarp();
         }
         if (probing) {
@@ -791,7 +864,7 @@ __global__ void __maxnreg__(96)
 #pragma unroll
           for (int qq = 0; qq < QH; ++qq) {
             const int qi = half * QH + qq;
-            const int b = score_bin(order_key(sc_[qq]), s.base[qi]);
+            const int b = dist_bin(sc_[qq], s.top[qi], s.base[qi]);
             red_add_shared_val_if(&s.hist[qi * kHistWords + (b >> 1)], 1u << ((b & 1) * 16),
                                   key <= s.pos[qi]);
           }
@@ -817,8 +890,7 @@ __global__ void __maxnreg__(96)
                   uint32_t A, Z;
                   find_crossing16<kBins / 32>(s.hist + qi * kHistWords, kBins, (uint32_t)r, bstar,
                                               A, Z);
-                  if (bstar > 0)
-                    t0 = key_to_float(static_cast<uint32_t>(s.base[qi] + bstar) << kBinShift);
+                  if (bstar > 0) t0 = bin_floor(bstar, s.top[qi], s.base[qi]);
                 }
               }
               if (lane == 0) s.tau[qi] = t0;
@@ -830,24 +902,37 @@ __global__ void __maxnreg__(96)
           }
           continue;
         }
-        const int i = step - np;  // main-pass tile index
-        if ((i & 3) == 0) {
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
-        }
         // Streaming selection: a passing lane appends to its own list.
         // Tiles wholly below every query's position need no causal compare.
-        const bool full_tile = (tile + 1) * kTileKeys <= minpos + 1;
+        if ((tile + 1) * kTileKeys <= minpos + 1) {
 #pragma unroll
-        for (int qq = 0; qq < QH; ++qq) {
-          const bool take = (full_tile || key <= s.pos[half * QH + qq]) && sc_[qq] >= tauR[qq];
-          st_global_u2_if(mylist + (qq * qstride + static_cast<uint32_t>(cnt[qq]) * 128u),
-                          __float_as_uint(sc_[qq]), static_cast<uint32_t>(key),
-                          take && cnt[qq] < rows_cap);
-          cnt[qq] += take ? 1 : 0;  // counts past rows_cap mark the list as overflowed
+          for (int qq = 0; qq < QH; ++qq) append_if(nxt[qq], sc_[qq], tauR[qq], key);
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq)
+            append_if(nxt[qq], sc_[qq], key <= s.pos[half * QH + qq] ? tauR[qq] : INFINITY, key);
+        }
+        const int i = step - np;  // main-pass tile index
+        if (probe && (i % kCheckTiles) == kCheckTiles - 1) {
+          // Each tile adds at most one row to a list, so a list may hold up
+          // to `room` rows now and still take every row of the tiles until
+          // the next check.  (Lists hold at least min(8, tiles) rows, so none
+          // can fill before the first check; the rescan launch's lists hold
+          // a row per tile and are not checked.)
+          const int room = ls.rows_cap - min(kCheckTiles, ntiles - 1 - i);
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) {
+            if (nxt[qq] - qlist(qq) > (int64_t)room * 128) {
+              tauR[qq] = INFINITY;
+              nxt[qq] = qlist(qq) + (int64_t)(ls.rows_cap + 1) * 128;
+            }
+          }
         }
       }
       if (!ok) break;
+      int cnt[QH];
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) cnt[qq] = static_cast<int>((nxt[qq] - qlist(qq)) >> 7);
       if (deferred) {
         // Leave the group's counts and histogram anchors for the selection
         // pass after this launch.
@@ -856,7 +941,8 @@ __global__ void __maxnreg__(96)
           if (half * QH + qq < nq) ls.counts_t(qb + half * QH + qq)[lrow] = cnt[qq];
         // (each half's lane-quarter-0 warp wrote these anchors itself)
         if (quarter == 0 && lane < QH && half * QH + lane < nq)
-          ls.anchor[qb + half * QH + lane] = s.base[half * QH + lane];
+          ls.anchor[qb + half * QH + lane] =
+              make_int2(s.base[half * QH + lane], __float_as_int(s.top[half * QH + lane]));
         ++gl;
         if (!(ok = ep_barrier(s, ephase, status))) break;
         continue;
@@ -870,6 +956,7 @@ __global__ void __maxnreg__(96)
         s.mpos[bsel * kMaxG + lane] = lane < G ? s.pos[lane] : -1;
         s.mrow[bsel * kMaxG + lane] = lane < G ? s.row[lane] : 0;
         s.mbase[bsel * kMaxG + lane] = lane < G ? s.base[lane] : 0;
+        s.mtop[bsel * kMaxG + lane] = lane < G ? s.top[lane] : 0.f;
         if (lane == 0) {
           s.selnq[bsel] = nq;
           s.selnext[bsel] = 0;
@@ -973,7 +1060,9 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm)
       if (napp < min(k, p + 1) || cmax > ls.rows_cap) {
         if (lane == 0) fail_out[atomicAdd(fail_count, 1)] = t;
       } else {
-        final_select(ls.list_t(t), ls.counts_t(t), ls.anchor[t], k, idx, val, selh);
+        const int2 an = ls.anchor[t];
+        final_select(ls.list_t(t), ls.counts_t(t), Anchor{__int_as_float(an.y), an.x}, k, idx,
+                     val, selh);
       }
     }
     __syncwarp();
@@ -1079,6 +1168,7 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
   fx.fail_in = a.fail_list;
   fx.fail_out = nullptr;
   fx.count = a.fail_count;
+  prof_count("#rescan_queries", a.fail_count, st);
   return launch_one<MH>(a, kmap, qmap, fx, fix_ls, st);
 }
 
@@ -1099,7 +1189,7 @@ size_t stream_cand_bytes(int grid, int64_t subcap, int m) {
 size_t stream_deferred_bytes(int T, int64_t subcap, int k) {
   const int rows = deferred_rows(k, subcap);
   return align256((size_t)T * rows * 128 * sizeof(uint2)) + align256((size_t)T * 128 * sizeof(int)) +
-         align256((size_t)T * sizeof(int));
+         align256((size_t)T * sizeof(int2));
 }
 
 int stream_deferred_rows(int k, int64_t subcap) { return deferred_rows(k, subcap); }

@@ -63,25 +63,30 @@ def check_heads(rep: Report, i, r_oracle, heads_gpu, m):
 
 def check_topk(rep: Report, i, I_oracle, idx_gpu, val_gpu, k, tokens=None):
     """Check one row of (idx, val) against oracle scores over `tokens`
-    (default: the prefix 0..n-1 with I_oracle indexed by token)."""
+    (sorted, distinct; default: the prefix 0..n-1 with I_oracle indexed by
+    token)."""
+    I_oracle = np.asarray(I_oracle, dtype=np.float64)
     n = len(I_oracle)
-    if tokens is None:
-        tokens = np.arange(n)
-    score_of = dict(zip((int(t) for t in tokens), I_oracle))
+    tokens = np.arange(n) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    idx_gpu = np.asarray(idx_gpu)
+    val_gpu = np.asarray(val_gpu)
     k_eff = min(k, n)
-    sel = [int(x) for x in idx_gpu if x >= 0]
-    if len(sel) != k_eff or len(set(sel)) != k_eff:
-        rep.fail(f"row {i}: {len(sel)} selected ({len(set(sel))} distinct), expected {k_eff}")
+    valid = idx_gpu >= 0
+    sel = idx_gpu[valid].astype(np.int64)
+    if len(sel) != k_eff or len(np.unique(sel)) != k_eff:
+        rep.fail(f"row {i}: {len(sel)} selected ({len(np.unique(sel))} distinct), expected {k_eff}")
         return
-    if any(x not in score_of for x in sel):
+    where = np.searchsorted(tokens, sel)
+    inside = (where < n) & (tokens[np.minimum(where, n - 1)] == sel)
+    if not inside.all():
         rep.fail(f"row {i}: selected token outside the candidate/prefix set")
         return
-    pad = [j for j, x in enumerate(idx_gpu) if x < 0]
-    if len(pad) != k - k_eff or not all(np.isneginf(val_gpu[j]) for j in pad):
+    pad = np.flatnonzero(~valid)
+    if len(pad) != k - k_eff or not np.all(np.isneginf(val_gpu[pad])):
         rep.fail(f"row {i}: bad padding")
     # values
-    sv = np.array([score_of[x] for x in sel])
-    gv = np.array([float(val_gpu[j]) for j, x in enumerate(idx_gpu) if x >= 0])
+    sv = I_oracle[where]
+    gv = val_gpu[valid].astype(np.float64)
     err = np.abs(gv - sv)
     if len(err):
         rep.max_val_err = max(rep.max_val_err, float((err / tol(sv)).max()))
@@ -89,22 +94,24 @@ def check_topk(rep: Report, i, I_oracle, idx_gpu, val_gpu, k, tokens=None):
             j = int(np.argmax(err - tol(sv)))
             rep.fail(f"row {i}: value of token {sel[j]} gpu={gv[j]:.7g} oracle={sv[j]:.7g}")
     # set compare with near-threshold allowance
-    _, ref_val = oracle.topk(np.asarray(I_oracle, dtype=np.float64), k)
-    order = np.lexsort((np.asarray(tokens), -(np.asarray(I_oracle) + 0.0)))[:k_eff]
-    ref = set(int(tokens[j]) for j in order)
-    g = set(sel)
+    order = np.lexsort((tokens, -(I_oracle + 0.0)))[:k_eff]
+    ref = set(tokens[order].tolist())
+    g = set(sel.tolist())
     if g != ref and k_eff < n:
         thr = I_oracle[order[-1]]
         for x in g ^ ref:
-            if abs(score_of[x] - thr) > tol(thr):
-                rep.fail(f"row {i}: token {x} I={score_of[x]:.7g} far from k-th {thr:.7g}")
+            sx = I_oracle[int(np.searchsorted(tokens, x))]
+            if abs(sx - thr) > tol(thr):
+                rep.fail(f"row {i}: token {x} I={sx:.7g} far from k-th {thr:.7g}")
                 return
         rep.topk_swaps += len(g - ref)
     # invariant: selected >= unselected (up to tolerance)
     if k_eff < n:
-        unsel = np.array([v for t, v in score_of.items() if t not in g])
-        if len(unsel) and sv.min() < unsel.max() - tol(unsel.max()):
-            rep.fail(f"row {i}: selected min {sv.min():.7g} < unselected max {unsel.max():.7g}")
+        unsel = np.ones(n, dtype=bool)
+        unsel[where] = False
+        umax = I_oracle[unsel].max()
+        if sv.min() < umax - tol(umax):
+            rep.fail(f"row {i}: selected min {sv.min():.7g} < unselected max {umax:.7g}")
 
 
 def check_misa_rows(wl, rows, idx, val, heads=None, r=None, Kbar=None, k=None, m=None,

@@ -95,10 +95,51 @@ def test_cpu_baseline_samples_the_oracle_on_all_cores_and_one_thread():
     assert out["cpu_model"]
 
 
-def test_mean_recall_of_two_selections():
+def test_recall_and_iou_rows_match_the_oracle_definition():
     import numpy as np
-    A = np.array([[1, 2, 3, -1], [5, 6, 7, 8], [-1, -1, -1, -1]])
-    D = np.array([[3, 2, 9, -1], [8, 7, 6, 5], [-1, -1, -1, -1]])
-    # row 0: {2,3} of {2,3,9}; row 1: all four; row 2 skipped (empty D)
-    assert abs(bench.mean_recall(A, D) - (2 / 3 + 1.0) / 2) < 1e-12
-    assert bench.mean_recall(D[2:], D[2:]) == 1.0
+    import torch
+
+    import oracle
+    A = np.array([[1, 2, 3, -1], [5, 6, 7, 8], [-1, -1, -1, -1], [4, 9, -1, -1]], np.int32)
+    D = np.array([[3, 2, 9, -1], [8, 7, 6, 5], [-1, -1, -1, -1], [1, 2, 3, 0]], np.int32)
+    rec, iou = bench.recall_iou_rows(torch.from_numpy(A), torch.from_numpy(D))
+    # row 2 is skipped (empty dense selection)
+    want = [oracle.recall_iou(A[i], D[i]) for i in (0, 1, 3)]
+    assert abs(rec - np.mean([r for r, _ in want])) < 1e-12
+    assert abs(iou - np.mean([u for _, u in want])) < 1e-12
+    # random rows of distinct indices with padding
+    rng = np.random.default_rng(0)
+    rows_a, rows_d = [], []
+    for _ in range(50):
+        n = int(rng.integers(1, 40))
+        a = rng.choice(60, size=n, replace=False)
+        d = rng.choice(60, size=int(rng.integers(1, 40)), replace=False)
+        rows_a.append(np.pad(a, (0, 40 - len(a)), constant_values=-1))
+        rows_d.append(np.pad(d, (0, 40 - len(d)), constant_values=-1))
+    A, D = np.array(rows_a, np.int32), np.array(rows_d, np.int32)
+    rec, iou = bench.recall_iou_rows(torch.from_numpy(A), torch.from_numpy(D))
+    want = [oracle.recall_iou(A[i], D[i]) for i in range(len(A))]
+    assert abs(rec - np.mean([r for r, _ in want])) < 1e-12
+    assert abs(iou - np.mean([u for _, u in want])) < 1e-12
+
+
+def test_split_prof_separates_counters_from_kernels():
+    kern, cnt = bench.split_prof({"score": (1.5, 2), "#rescan_queries": (0.0, 7),
+                                  "select": (0.5, 1)})
+    assert kern == {"score": (1.5, 2), "select": (0.5, 1)}
+    assert cnt == {"rescan_queries": 7}
+
+
+def test_roofline_uses_the_burst_peak_for_prefill_and_hbm_for_decode():
+    from misa_synth import make_workload
+    wl = make_workload(seq_lens=[4096], queries="all", H=8, B=64, m=8, k=16, seed=1)
+    peaks = {"bf16": 1600.0, "bf16_sustained": 1400.0, "hbm_gbs": 6500.0, "source": "test"}
+    r = bench.roofline_of(wl, 2.0, 1, True, peaks, {"sm_mhz": 1800.0}, "none")
+    flops = 2 * 8 * 128 * wl.pairs
+    assert abs(r["achieved"] - flops / 2e-3 / 1e12) < 1e-9
+    assert r["peak"] == 1600.0 and abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
+    assert abs(r["frac_of_sustained"] - r["achieved"] / 1400.0) < 1e-12
+    wl2 = make_workload(seq_lens=[1000, 500], queries=3, H=8, B=64, m=8, k=16, seed=1)
+    r2 = bench.roofline_of(wl2, 0.01, 1, False, peaks, {}, "none")
+    abytes = (1000 + 500) * 256 + 4 * wl2.pairs
+    assert r2["bound"] == "hbm" and abs(r2["achieved"] - abytes / 1e-5 / 1e9) < 1e-6

@@ -205,6 +205,8 @@ def test_stream_probe_overestimate_goes_through_fixup():
     misa.profile_enable(False)
     status_ok()
     assert "score_fixup" in prof
+    # the queries with the overestimating sample (long enough to be probed)
+    assert prof["#rescan_queries"][1] > 1000
     si, sv = ix.idx.clone(), ix.val.clone()
     dbg = torch.empty((wl.T, L), dtype=torch.float32, device="cuda")
     misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, Kd, wl.k, ix.idx, ix.val, ix.ws, dbg)
@@ -242,3 +244,38 @@ def test_hier_prefill_streamed_candidates_then_rerank():
                            m=wl.m).assert_ok()
     parity.check_rerank_rows(wl, rows, ix.cand[sel].cpu().numpy(), ix.idx[sel].cpu().numpy(),
                              ix.val[sel].cpu().numpy()).assert_ok()
+
+
+def test_stream_dense_rescan_at_prefill_size():
+    # The probe-overestimate pattern with all heads (the dense indexer) over a
+    # 32K prefill: most queries fail their sampled threshold and go through
+    # the rescan launch, which must still give the exact top-k.
+    L, H, d = 32768, 32, 128
+    wl = make_workload(seq_lens=[L], queries="all", H=H, B=128, m=H, k=2048, seed=8,
+                       needles=False)
+    K = np.zeros((L, d), np.float32)
+    K[:, 0] = 1.0
+    s = np.arange(L)
+    high = ((s // 128) % 8 == 4) & (s % 2 == 0)
+    K[high, 0] = 10.0
+    K[:, 1] = (s % 7) * 0.125  # distinct scores inside a tile
+    rng = np.random.default_rng(8)
+    q = np.zeros((L, H, d), np.float32)
+    q[:, :, 0] = 1.0
+    q[:, :, 1] = rng.integers(0, 3, size=(L, H)) * 0.5
+    w = rng.uniform(0.05, 0.2, size=(L, H)).astype(np.float32)
+    wl = dataclasses.replace(wl, K_bits=f32_to_bf16_bits(K), q_bits=f32_to_bf16_bits(q), w=w)
+    prob, Kd, qd, wd = dev(wl)
+    ix = misa.Indexer(prob, m=8, k=wl.k)
+    misa.profile_enable(True)
+    ix.dense(qd, wd, Kd)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert "topk" not in prof
+    assert prof["#rescan_queries"][1] > L // 4
+    invariants(wl, ix.idx)
+    rows = [0, 2047, 2048, 2049, 9000, 20000, L - 2, L - 1]
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_dense_rows(wl, rows, ix.idx[sel].cpu().numpy(),
+                            ix.val[sel].cpu().numpy()).assert_ok()
