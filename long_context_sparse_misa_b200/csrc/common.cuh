@@ -315,6 +315,21 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, 
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
 }
 
+// acc = {a0, a1} += {w0, w1} * {r0, r1} (one packed fp32 FMA; the weights
+// come as a 64-bit pair and the accumulators stay packed between calls).
+__device__ __forceinline__ void ffma2_acc(uint64_t& acc, uint64_t w, float r0, float r1) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(r0), "f"(r1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(r));
+}
+
+// a0 + a1 of a packed pair.
+__device__ __forceinline__ float sum_pair(uint64_t acc) {
+  float a0, a1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+  return a0 + a1;
+}
+
 // Head-weighted ReLU sum of one query's MH accumulator columns, the one
 // summation order every scoring kernel uses (so all paths agree bit for bit):
 // even heads into a0, odd heads into a1 (one packed FMA per pair), then

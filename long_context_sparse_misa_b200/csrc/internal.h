@@ -140,6 +140,7 @@ struct ScoreArgs {
   int64_t ld;
   int max_tiles;          // host bound on key tiles per group
   bool direct = false;    // gather mode without a plan: group i is query row i
+  bool row_by_group = false;  // groups of one query each; group i writes row i of I
 };
 int launch_score(const ScoreArgs& a, cudaStream_t st);
 
@@ -180,8 +181,12 @@ int score_group_size(int m);
 // For query rows [q_lo, q_hi): select the top-k of I row (t - q_lo).
 // Contiguous mode (tok == nullptr): elements 0..q_pos[t], token = element index.
 // Token mode: elements 0..n_fixed-1 with token tok[t * n_fixed + e] (< 0 = absent).
+// rows_list / rows_count (device, optional): row i of I belongs to query
+// rows_list[i] for i < *rows_count; rows past the count are skipped (the
+// grid still covers q_hi - q_lo rows).
 int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32_t* tok,
                 int n_fixed, int q_lo, int q_hi, int k, int32_t* idx, float* val,
-                cudaStream_t st);
+                cudaStream_t st, const int32_t* rows_list = nullptr,
+                const int* rows_count = nullptr);
 
 }  // namespace misa

@@ -15,9 +15,11 @@
 // accumulators of 128 rows x 128 blocks (all 512 columns).  The fp32 pooled
 // keys enter as a bf16 pair hi = bf16(Kbar), lo = bf16(Kbar - hi)
 // accumulated into the same fp32 accumulator, which keeps ~16 mantissa bits
-// of the pooled keys.  Epilogue warps own one row of each accumulator per
-// lane, so the block-axis ReLU-sum is inside the thread; an accumulator is
-// released as soon as it is copied to registers.  The causal partial block
+// of the pooled keys.  Eight epilogue warps, two per TMEM lane quarter:
+// each owns one row of every accumulator per lane and half of each chunk's
+// columns, so the block-axis ReLU-sum is inside the thread (the two halves
+// are added in shared memory); an accumulator is released as soon as both
+// halves are copied to registers.  The causal partial block
 // of every key position (the running mean of its block up to that key) is
 // computed beforehand by one warp per pooled block, so each query only
 // reads its row.  Persistent: one CTA per SM walks its groups; the next
@@ -29,7 +31,9 @@
 namespace misa {
 namespace {
 
-constexpr int kThreads = 192;          // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEpiWarps = 8;           // two per TMEM lane quarter, one per half of a chunk
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kRows = 512;             // q rows per CTA (4 accumulators of 128)
 constexpr int kChunk = 128;            // pooled blocks per chunk (accumulator columns)
 constexpr int kStages = 2;             // each stage: one of hi/lo for one chunk (2048 MMA cycles)
@@ -39,13 +43,15 @@ constexpr int kQHalfBytes = kRows * 128;              // 64 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kMaxG = 16;                             // queries per group
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kRows * 4 /*r*/ +
-                           kMaxG * kD * 4 /*pm*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
+                           2 * kRows * 4 /*racc*/ + kMaxG * kD * 4 /*pm*/ + kMaxG * 4 * 2 +
+                           16 * 8 + 16;
 
 struct Smem {
   uint8_t* q;
   uint8_t* k;
-  float* r;   // [kRows] router scores of the group
-  float* pm;  // [kMaxG][128] running block means at the group's query positions
+  float* r;     // [kRows] router scores of the group
+  float* racc;  // [2][kRows] block-axis ReLU sums of each half of the chunks
+  float* pm;    // [kMaxG][128] running block means at the group's query positions
   int* pos;
   int* flags;
   uint64_t* full;
@@ -66,7 +72,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.q = p;
   s.k = p + kQBytes;
   s.r = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
-  s.pm = s.r + kRows;
+  s.racc = s.r + kRows;
+  s.pm = s.racc + 2 * kRows;
   s.pos = reinterpret_cast<int*>(s.pm + kMaxG * kD);
   s.flags = s.pos + kMaxG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.empty[i], 1);
     }
     mbar_init(s.tfull, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&s.tempty[i], 4);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.tempty[i], kEpiWarps);
     mbar_init(s.qfull, 1);
     mbar_init(s.qempty, 1);
     mbar_init(s.drain, 1);
@@ -264,8 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;            // 0..127
+    // Warp e = warp - 2: TMEM lane quarter warp % 4, columns ch*64 .. ch*64+63
+    // of every 128-block chunk (ch = e / 4); each thread sums the ReLU of its
+    // row's visible columns, and the two halves are added in shared memory.
+    const int et = threadIdx.x - 64;            // 0..kEpiThreads-1
     const int quarter = warp & 3;
+    const int ch = (warp - 2) >> 2;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int cc = 0;
     bool ok = true;
@@ -274,11 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int seq = grp.x, qb = grp.y, nq = grp.z - grp.y;
       if (grp.w < 0 || nq <= 0) {
         // no valid query: deterministic padding for every row of the group
-        for (int i = et; i < nq * m; i += 128) {
+        for (int i = et; i < nq * m; i += kEpiThreads) {
           heads[(int64_t)qb * m + i] = -1;
           w_r[(int64_t)qb * m + i] = 0.f;
         }
-        for (int i = et; i < nq * m * (kD / 8); i += 128)
+        for (int i = et; i < nq * m * (kD / 8); i += kEpiThreads)
           reinterpret_cast<uint4*>(q_r + (int64_t)qb * m * kD)[i] = make_uint4(0, 0, 0, 0);
         continue;
       }
@@ -292,10 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         s.pos[et] = p;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       // The queries' running block means (partial block), staged for the
       // head rows of each query (coalesced 16-byte loads).
-      for (int i = et; i < nq * (kD / 4); i += 128) {
+      for (int i = et; i < nq * (kD / 4); i += kEpiThreads) {
         const int qi = i / (kD / 4), c4 = i - qi * (kD / 4);
         const int p = s.pos[qi];
         if (p >= 0 && (p + 1) % B != 0)
@@ -304,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
-      // of every accumulator.
+      // of every accumulator, columns ch*64 .. ch*64+63 of each chunk.
       float acc[NSUB];
       int lim[NSUB];
 #pragma unroll
@@ -313,27 +324,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = sub * 128 + quarter * 32 + lane;
         const int qi = row / H;
         const int p = (row < ROWS && qi < nq) ? s.pos[qi] : -1;
-        lim[sub] = (p + 1) / B;  // number of full blocks visible to this row
+        lim[sub] = (p + 1) / B - ch * 64;  // full blocks visible, from this half's first column
       }
       for (int c = 0; c < nchunks && ok; ++c, ++cc) {
         if (!(ok = warp_wait(s.tfull, cc & 1, s.abort, status))) break;
         tc_fence_after();
 #pragma unroll
         for (int sub = 0; sub < NSUB; ++sub) {
-          float v[4][32];
+          float v[2][32];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) tmem_ld32(lane_addr + sub * kChunk + j * 32, v[j]);
+          for (int j = 0; j < 2; ++j)
+            tmem_ld32(lane_addr + sub * kChunk + ch * 64 + j * 32, v[j]);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) reg_fence32(v[j]);
+          for (int j = 0; j < 2; ++j) reg_fence32(v[j]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s.tempty[sub]);
-          const int nvis = lim[sub] - c * kChunk;  // visible columns of this chunk
-          if (nvis >= kChunk) {
+          const int nvis = lim[sub] - c * kChunk;  // visible columns of this half-chunk
+          if (nvis >= 64) {
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int x = 0; x < 32; x += 2) {
                 a0 += fmaxf(v[j][x], 0.f);
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else if (nvis > 0) {
             float a0 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int x = 0; x < 32; ++x)
                 if (j * 32 + x < nvis) a0 += fmaxf(v[j][x], 0.f);
@@ -352,17 +364,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // s.pm complete
-
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
         const int row = sub * 128 + quarter * 32 + lane;
-        if (row >= ROWS) continue;
+        if (row < ROWS) s.racc[ch * kRows + row] = acc[sub];
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");  // s.pm, s.racc complete
+
+      for (int row = et; row < ROWS; row += kEpiThreads) {
         const int qi = row / H, h = row - qi * H;
         float r = -INFINITY;
         if (qi < nq && s.pos[qi] >= 0) {
           const int p = s.pos[qi];
-          float total = acc[sub];
+          float total = s.racc[row] + s.racc[kRows + row];
           if ((p + 1) % B != 0) {
             const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)(qb + qi) * H + h) * kD);
             const float* Pq = s.pm + qi * kD;  // running block mean at p
@@ -390,12 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         s.r[row] = r;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       // Top-m per query by (r desc, head asc): rank of each head.
-#pragma unroll
-      for (int sub = 0; sub < NSUB; ++sub) {
-        const int row = sub * 128 + quarter * 32 + lane;
-        if (row >= ROWS) continue;
+      for (int row = et; row < ROWS; row += kEpiThreads) {
         const int qi = row / H, h = row - qi * H;
         if (qi >= nq) continue;
         const int64_t t = qb + qi;
@@ -425,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kD / 8; ++i) dst[i] = __ldg(src + i);
         }
       }
-      // s.pos and s.r are rewritten by the next group
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // s.pos, s.racc and s.r are rewritten by the next group
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
     }
   }
 

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
                  const int32_t* __restrict__ cand, int k_cand, const int4* __restrict__ groups,
                  const int* __restrict__ group_count, int tiles_per_split, int q_lo,
                  float* __restrict__ I, int64_t ld, int64_t total_keys, uint32_t* status,
-                 const int32_t* __restrict__ qo, int S, int direct_T) {
+                 const int32_t* __restrict__ qo, int S, int direct_T, int row_by_group) {
   pdl_wait_then_release();
   constexpr int G = GATHER ? 1 : kMaxN / MH;
   static_assert(G * MH <= kMaxN, "group too wide");
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
         if (pos < 0 || pos >= L) pos = -1;
       }
       s.pos[qi] = pos;
-      s.row[qi] = qb + qi - q_lo;
+      // row_by_group: one query per group, written to row gi (a list of queries)
+      s.row[qi] = row_by_group ? gi + qi : qb + qi - q_lo;
     }
   }
   tc_fence_before();
@@ -356,12 +357,12 @@ int launch_one(const ScoreArgs& a, const CUtensorMap& kmap, const CUtensorMap& q
   auto kern = score_kernel<MH, GATHER>;
   int rc = set_smem_limit((const void*)kern, kSmemBytes);
   if (rc) return rc;
-  ProfScope ps(GATHER ? "rerank_score" : "score", st);
+  ProfScope ps(GATHER ? "rerank_score" : (a.row_by_group ? "rescan_score" : "score"), st);
   return cuda_fail(launch_pdl(kern, grid, dim3(threads_for(GATHER)), kSmemBytes, st, kmap, qmap, a.K,
                               a.wsel, a.p->q_pos, a.p->key_offsets, a.cand, a.k_cand, a.groups,
                               a.group_count, tps, a.q_lo, a.I, a.ld, a.p->total_keys,
                               status_ptr(), a.p->query_offsets, a.p->num_seqs,
-                              a.direct ? a.p->num_queries : 0),
+                              a.direct ? a.p->num_queries : 0, a.row_by_group ? 1 : 0),
                    "score_kernel");
 }
 

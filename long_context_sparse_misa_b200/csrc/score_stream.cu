@@ -94,6 +94,7 @@ constexpr int kProbeStride = 24;                 // probe every 24th tile ...
 constexpr int kProbeOff = 12;                    // ... starting at tile 12
 constexpr int kProbeMinTiles = 16;               // only prefixes of >= 2048 keys
 constexpr int kCheckTiles = 8;                   // list capacity checked every 8 tiles
+constexpr int kRescanCap = 128;                  // failed queries rescanned as score rows
 
 static_assert(kSelBins >= kBins, "final-select histogram");
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kN * 4 /*w*/ +
@@ -220,26 +221,31 @@ __device__ __forceinline__ float bin_floor(int b, float top, int base) {
 
 // Columns C*16 .. C*16+15 of a warp's 64: the head-weighted ReLU sums in the
 // order of relu_wsum (even heads into a0, odd into a1, then a0 + a1), with
-// a query's running sums carried across chunks when it spans several.  The
-// halved weights come four at a time (one 16-byte shared load).
+// a query's running sums acc = {a0, a1} carried across chunks when it spans
+// several.  The halved weights come four at a time (one 16-byte shared load
+// into two 64-bit pairs), so neither operand of the packed FMA is repacked.
 template <int MH, int C, int QH>
-__device__ __forceinline__ void chunk_wsum(const float (&v)[16], const float* wcol, float& a0,
-                                           float& a1, float (&sc)[QH]) {
+__device__ __forceinline__ void chunk_wsum(const float (&v)[16], const float* wcol,
+                                           uint64_t& acc, float (&sc)[QH], int tile_dep) {
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     constexpr int kBase = C * 16;
     const int col = kBase + 4 * p;
-    const float4 w4 = *reinterpret_cast<const float4*>(wcol + col);
+    // The load is not volatile, so it may be scheduled early within the
+    // tile; `tile_dep` (unused by the instruction) ties it to this tile so it
+    // is never hoisted out of the tile loop or above the barrier after which
+    // a group's weights are written.
+    uint64_t wlo, whi;
+    asm("ld.shared.v2.b64 {%0, %1}, [%2];"
+        : "=l"(wlo), "=l"(whi)
+        : "r"(smem_u32(wcol + col)), "r"(tile_dep));
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c2 = col + 2 * h;
-      if (c2 % MH == 0) {
-        a0 = 0.f;
-        a1 = 0.f;
-      }
+      if (c2 % MH == 0) acc = 0ull;  // {+0, +0}
       const float c0 = v[4 * p + 2 * h], c1 = v[4 * p + 2 * h + 1];
-      ffma2(a0, a1, h ? w4.z : w4.x, h ? w4.w : w4.y, c0 + fabsf(c0), c1 + fabsf(c1));
-      if ((c2 + 2) % MH == 0) sc[c2 / MH] = a0 + a1;
+      ffma2_acc(acc, h ? whi : wlo, c0 + fabsf(c0), c1 + fabsf(c1));
+      if ((c2 + 2) % MH == 0) sc[c2 / MH] = sum_pair(acc);
     }
   }
 }
@@ -518,6 +524,13 @@ __device__ __forceinline__ int probe_tiles(bool probe, int ntiles) {
   return np < kProbeMaxTiles ? np : kProbeMaxTiles;
 }
 
+// MMA width N: the group's 256 (query, head) columns, or in the rescan
+// launch (one query per group) only that query's MH heads (at least 16).
+template <int MH>
+__device__ __forceinline__ int mma_cols(bool probe) {
+  return probe ? kN : (MH < 16 ? 16 : MH);
+}
+
 // Candidate list of (buffer b, query slot q) of this CTA: rows_cap rows of 128.
 // Deferred selection (anchor != nullptr): one list per query row t instead,
 // [T][rows_cap][128] with counts [T][128] and the query's histogram anchor,
@@ -675,9 +688,10 @@ __global__ void __maxnreg__(96)
         const int ntiles = (grp.w + kTileKeys) / kTileKeys;
         const int np = probe_tiles(probe, ntiles);
         if (!(ok = mbar_wait(s.qempty, (gl & 1) ^ 1, s.abort, status))) break;
-        mbar_arrive_expect_tx(s.qfull, kQBytes);
+        const int qrows = (mma_cols<MH>(probe) + 31) / 32 * 32;  // query rows the MMAs read
+        mbar_arrive_expect_tx(s.qfull, 2u * qrows * 128u);
         for (int h = 0; h < 2; ++h)
-          for (int r0 = 0; r0 < kN; r0 += 32)
+          for (int r0 = 0; r0 < qrows; r0 += 32)
             tma_load_2d(&qmap, s.qfull, s.q + h * kQHalfBytes + r0 * 128, h * 64,
                         grp.y * MH + r0);
         ++gl;
@@ -700,7 +714,7 @@ __global__ void __maxnreg__(96)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kTileKeys, kN);
+      const uint32_t idesc = idesc_bf16_f32(kTileKeys, mma_cols<MH>(probe));
       const uint32_t q_addr = smem_u32(s.q);
       int it = 0, tb = 0, gl = 0;
       bool ok = true;
@@ -802,132 +816,178 @@ __global__ void __maxnreg__(96)
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
 
-      for (int step = 0; step < np + ntiles; ++step, ++tb) {
-        const bool probing = step < np;
-        const int tile = probing ? kProbeOff + kProbeStride * step : step - np;
+      // One tile: wait for its accumulators, read the warp's 64 columns in
+      // four 16-column TMEM loads (each issued before the previous chunk is
+      // summed, so the load latency overlaps the arithmetic; the buffer is
+      // released after the last load) and form this lane's score of each of
+      // the warp's queries.  The tile loops below are specialised (probe
+      // tiles, full main-pass tiles in runs of kCheckTiles, the diagonal
+      // tiles) so that no per-tile branch sits around this body.
+      // (In the rescan launch the MMAs fill only the first query's columns;
+      // the other columns hold stale values, read but never used: those query
+      // slots are padding, which never appends.)
+      auto tile_scores = [&](float (&sc_)[QH]) -> bool {
         const int buf = tb & 1;
-        if (!(ok = warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status))) break;
+        if (!warp_wait(&s.tfull[buf], (tb >> 1) & 1, s.abort, status)) return false;
         tc_fence_after();
-        // The warp's 64 columns in four 16-column TMEM loads, each issued
-        // before the previous chunk is summed, so the load latency overlaps
-        // the arithmetic; the buffer is released after the last load.
         const uint32_t taddr = lane_addr + buf * kN + half * kColsPerWarp;
         const float* wcol = s.w + half * kColsPerWarp;
-        float sc_[QH];
-        float a0 = 0.f, a1 = 0.f;
+        uint64_t acc = 0ull;
         float vA[16], vB[16];
         tmem_ld16(taddr, vA);
         tmem_wait_ld();
         reg_fence16(vA);
         tmem_ld16(taddr + 16, vB);
-        chunk_wsum<MH, 0>(vA, wcol, a0, a1, sc_);
+        chunk_wsum<MH, 0>(vA, wcol, acc, sc_, tb);
         tmem_wait_ld();
         reg_fence16(vB);
         tmem_ld16(taddr + 32, vA);
-        chunk_wsum<MH, 1>(vB, wcol, a0, a1, sc_);
+        chunk_wsum<MH, 1>(vB, wcol, acc, sc_, tb);
         tmem_wait_ld();
         reg_fence16(vA);
         tmem_ld16(taddr + 48, vB);
-        chunk_wsum<MH, 2>(vA, wcol, a0, a1, sc_);
+        chunk_wsum<MH, 2>(vA, wcol, acc, sc_, tb);
         tmem_wait_ld();
         reg_fence16(vB);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tempty[buf]);
-        chunk_wsum<MH, 3>(vB, wcol, a0, a1, sc_);
-        const int key = tile * kTileKeys + lrow;
-        if (step == 0) {
-          // Anchor every query's histogram on the range of its first tile.
+        chunk_wsum<MH, 3>(vB, wcol, acc, sc_, tb);
+        ++tb;
+        return true;
+      };
+      // Anchor every query's histogram on the range of its first scored tile.
+      auto anchor = [&](const float (&sc_)[QH], int key) -> bool {
 #pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
-            const int qi = half * QH + qq;
-            const bool v = key <= s.pos[qi];
-            const uint32_t kk = order_key(sc_[qq]);
-            const uint32_t hi = __reduce_max_sync(0xffffffffu, v ? kk : 0u);
-            const uint32_t lo = __reduce_min_sync(0xffffffffu, v ? kk : 0xFFFFFFFFu);
-            if (lane == 0) {
-              atomicMax(&s.maxkey[qi], hi);
-              atomicMin(&s.minkey[qi], lo);
+        for (int qq = 0; qq < QH; ++qq) {
+          const int qi = half * QH + qq;
+          const bool v = key <= s.pos[qi];
+          const uint32_t kk = order_key(sc_[qq]);
+          const uint32_t hi = __reduce_max_sync(0xffffffffu, v ? kk : 0u);
+          const uint32_t lo = __reduce_min_sync(0xffffffffu, v ? kk : 0xFFFFFFFFu);
+          if (lane == 0) {
+            atomicMax(&s.maxkey[qi], hi);
+            atomicMin(&s.minkey[qi], lo);
+          }
+        }
+        if (!ep_barrier(s, ephase, status)) return false;
+        // every warp of a half writes the same anchors for its queries
+        if (lane < QH) {
+          const Anchor a = make_anchor(s.maxkey[half * QH + lane], s.minkey[half * QH + lane]);
+          s.base[half * QH + lane] = a.base;
+          s.top[half * QH + lane] = a.top;
+        }
+        __syncwarp();
+        return true;
+      };
+      // Streaming selection: a passing lane appends to its own list.  Tiles
+      // wholly below every query's position need no causal compare.
+      auto append_full = [&](const float (&sc_)[QH], int key) {
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) append_if(nxt[qq], sc_[qq], tauR[qq], key);
+      };
+      auto append_causal = [&](const float (&sc_)[QH], int key) {
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq)
+          append_if(nxt[qq], sc_[qq], key <= s.pos[half * QH + qq] ? tauR[qq] : INFINITY, key);
+      };
+      // After main-pass tiles 0..i-1: each tile adds at most one row to a
+      // list, so a list may hold up to `room` rows now and still take every
+      // row of the tiles until the next check.  (Lists hold at least
+      // min(8, tiles) rows, so none can fill before the first check; the
+      // rescan launch's lists hold a row per tile and are not checked.)
+      auto check_room = [&](int i) {
+        if (!probe || i >= ntiles) return;
+        const int room = ls.rows_cap - min(kCheckTiles, ntiles - i);
+        // (the list starts are recomputed here rather than kept in registers
+        // across the tile loops: the volatile copy keeps the compiler from
+        // hoisting them)
+        int64_t qs;
+        asm volatile("mov.b64 %0, %1;" : "=l"(qs) : "l"(qstride));
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) {
+          const uint2* start = mylist + qq * qs;
+          if (nxt[qq] - start > (int64_t)room * 128) {
+            tauR[qq] = INFINITY;
+            nxt[qq] = const_cast<uint2*>(start) + (int64_t)(ls.rows_cap + 1) * 128;
+          }
+        }
+      };
+
+      // ---- probe tiles (kProbeOff + kProbeStride * j): histogram only
+      for (int step = 0; step < np; ++step) {
+        float sc_[QH];
+        if (!(ok = tile_scores(sc_))) break;
+        const int key = (kProbeOff + kProbeStride * step) * kTileKeys + lrow;
+        if (step == 0 && !(ok = anchor(sc_, key))) break;
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) {
+          const int qi = half * QH + qq;
+          const int b = dist_bin(sc_[qq], s.top[qi], s.base[qi]);
+          red_add_shared_val_if(&s.hist[qi * kHistWords + (b >> 1)], 1u << ((b & 1) * 16),
+                                key <= s.pos[qi]);
+        }
+      }
+      if (!ok) break;
+      if (np > 0) {
+        // Starting thresholds from the sample: the bin holding the r-th best
+        // sampled score, r = k*f + 4*sqrt(k*f) + 1 (f: sampled share of the
+        // query's prefix).  Verified at the end of the group.
+        if (!(ok = ep_barrier(s, ephase, status))) break;
+        for (int qi = e; qi < G; qi += kEpiWarps) {
+          const int n = s.pos[qi] + 1;
+          int ns = 0;
+          for (int j = lane; j < np; j += 32) {
+            const int rem = n - (kProbeOff + kProbeStride * j) * kTileKeys;
+            ns += rem <= 0 ? 0 : (rem > kTileKeys ? kTileKeys : rem);
+          }
+          ns = __reduce_add_sync(0xffffffffu, ns);
+          float t0 = s.pos[qi] >= 0 ? -INFINITY : INFINITY;
+          if (n > k && ns > 0) {
+            const float ks = (float)k * (float)ns / (float)n;
+            const int r = (int)ceilf(ks + 4.f * sqrtf(ks)) + 1;
+            if (r <= ns) {
+              int bstar;
+              uint32_t A, Z;
+              find_crossing16<kBins / 32>(s.hist + qi * kHistWords, kBins, (uint32_t)r, bstar, A,
+                                          Z);
+              if (bstar > 0) t0 = bin_floor(bstar, s.top[qi], s.base[qi]);
             }
           }
-          if (!(ok = ep_barrier(s, ephase, status))) break;
-          // every warp of a half writes the same anchors for its queries
-          if (lane < QH) {
-            const Anchor a = make_anchor(s.maxkey[half * QH + lane], s.minkey[half * QH + lane]);
-            s.base[half * QH + lane] = a.base;
-            s.top[half * QH + lane] = a.top;
-          }
-          __syncwarp();
+          if (lane == 0) s.tau[qi] = t0;
+          for (int b = lane; b < kHistWords; b += 32) s.hist[qi * kHistWords + b] = 0u;
         }
-        if (probing) {
-          // Probe: histogram every sampled score (no appends).
+        if (!(ok = ep_barrier(s, ephase, status))) break;
 #pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
-            const int qi = half * QH + qq;
-            const int b = dist_bin(sc_[qq], s.top[qi], s.base[qi]);
-            red_add_shared_val_if(&s.hist[qi * kHistWords + (b >> 1)], 1u << ((b & 1) * 16),
-                                  key <= s.pos[qi]);
-          }
-          if (step == np - 1) {
-            // Starting thresholds from the sample: the bin holding the r-th
-            // best sampled score, r = k*f + 4*sqrt(k*f) + 1 (f: sampled share
-            // of the query's prefix).  Verified at the end of the group.
-            if (!(ok = ep_barrier(s, ephase, status))) break;
-            for (int qi = e; qi < G; qi += kEpiWarps) {
-              const int n = s.pos[qi] + 1;
-              int ns = 0;
-              for (int j = lane; j < np; j += 32) {
-                const int rem = n - (kProbeOff + kProbeStride * j) * kTileKeys;
-                ns += rem <= 0 ? 0 : (rem > kTileKeys ? kTileKeys : rem);
-              }
-              ns = __reduce_add_sync(0xffffffffu, ns);
-              float t0 = s.pos[qi] >= 0 ? -INFINITY : INFINITY;
-              if (n > k && ns > 0) {
-                const float ks = (float)k * (float)ns / (float)n;
-                const int r = (int)ceilf(ks + 4.f * sqrtf(ks)) + 1;
-                if (r <= ns) {
-                  int bstar;
-                  uint32_t A, Z;
-                  find_crossing16<kBins / 32>(s.hist + qi * kHistWords, kBins, (uint32_t)r, bstar,
-                                              A, Z);
-                  if (bstar > 0) t0 = bin_floor(bstar, s.top[qi], s.base[qi]);
-                }
-              }
-              if (lane == 0) s.tau[qi] = t0;
-              for (int b = lane; b < kHistWords; b += 32) s.hist[qi * kHistWords + b] = 0u;
-            }
-            if (!(ok = ep_barrier(s, ephase, status))) break;
-#pragma unroll
-            for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
-          }
-          continue;
+        for (int qq = 0; qq < QH; ++qq) tauR[qq] = s.tau[half * QH + qq];
+      }
+
+      // ---- main pass over tiles 0..ntiles-1
+      const int nfull = min(ntiles, (minpos + 1) / kTileKeys);  // tiles below every position
+      int i = 0;
+      if (np == 0 && ntiles > 0) {
+        // no probe: the first main tile anchors the histograms
+        float sc_[QH];
+        if (!(ok = tile_scores(sc_))) break;
+        const int key = lrow;
+        if (!(ok = anchor(sc_, key))) break;
+        if (nfull > 0) append_full(sc_, key); else append_causal(sc_, key);
+        i = 1;
+      }
+      while (ok && i < nfull) {
+        const int iend = min(nfull, (i / kCheckTiles + 1) * kCheckTiles);
+        for (; i < iend; ++i) {
+          float sc_[QH];
+          if (!(ok = tile_scores(sc_))) break;
+          append_full(sc_, i * kTileKeys + lrow);
         }
-        // Streaming selection: a passing lane appends to its own list.
-        // Tiles wholly below every query's position need no causal compare.
-        if ((tile + 1) * kTileKeys <= minpos + 1) {
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq) append_if(nxt[qq], sc_[qq], tauR[qq], key);
-        } else {
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq)
-            append_if(nxt[qq], sc_[qq], key <= s.pos[half * QH + qq] ? tauR[qq] : INFINITY, key);
-        }
-        const int i = step - np;  // main-pass tile index
-        if (probe && (i % kCheckTiles) == kCheckTiles - 1) {
-          // Each tile adds at most one row to a list, so a list may hold up
-          // to `room` rows now and still take every row of the tiles until
-          // the next check.  (Lists hold at least min(8, tiles) rows, so none
-          // can fill before the first check; the rescan launch's lists hold
-          // a row per tile and are not checked.)
-          const int room = ls.rows_cap - min(kCheckTiles, ntiles - 1 - i);
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
-            if (nxt[qq] - qlist(qq) > (int64_t)room * 128) {
-              tauR[qq] = INFINITY;
-              nxt[qq] = qlist(qq) + (int64_t)(ls.rows_cap + 1) * 128;
-            }
-          }
-        }
+        if (ok && i % kCheckTiles == 0) check_room(i);
+      }
+      for (; ok && i < ntiles; ++i) {
+        float sc_[QH];
+        if (!(ok = tile_scores(sc_))) break;
+        append_causal(sc_, i * kTileKeys + lrow);
+        if (i % kCheckTiles == kCheckTiles - 1) check_room(i + 1);
       }
       if (!ok) break;
       int cnt[QH];
@@ -1081,11 +1141,14 @@ int deferred_rows(int k, int64_t rows_full) {
 }
 
 // Candidate storage (one workspace region, 256-byte aligned parts): the main
-// pass's lists [grid][2][G][rows_main][128] and counts, then the rescan's
-// lists [grid][2][1][rows_full][128] and counts.
+// pass's lists [grid][2][G][rows_main][128] and counts, the in-kernel
+// rescan's lists [grid][2][1][rows_full][128] and counts, then the
+// split rescan's score rows [kRescanCap][row_ld] fp32, its one-query groups
+// int4 [kRescanCap] and two counters {queries rescanned by rows, rest}.
 struct CandLayout {
   int rows_main, rows_full;
-  size_t main_lists, main_counts, fix_lists, fix_counts;
+  int64_t row_ld;
+  size_t main_lists, main_counts, fix_lists, fix_counts, rescan_rows, rescan_groups;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1094,11 +1157,36 @@ CandLayout cand_layout(int grid, int64_t rows_full, int G) {
   CandLayout c;
   c.rows_full = (int)rows_full;
   c.rows_main = (int)(rows_full < kRowsCap ? rows_full : kRowsCap);
+  c.row_ld = rows_full * kTileKeys;
   c.main_lists = align256((size_t)grid * 2 * G * c.rows_main * 128 * sizeof(uint2));
   c.main_counts = align256((size_t)grid * 2 * G * 128 * sizeof(int));
   c.fix_lists = align256((size_t)grid * 2 * c.rows_full * 128 * sizeof(uint2));
   c.fix_counts = align256((size_t)grid * 2 * 128 * sizeof(int));
+  c.rescan_rows = align256((size_t)kRescanCap * c.row_ld * sizeof(float));
+  c.rescan_groups = align256((size_t)kRescanCap * sizeof(int4) + 16);
   return c;
+}
+
+// The first kRescanCap failed queries become one-query groups for the split
+// rescan (the decode-path scorer spreads each over several CTAs, then the
+// top-k selects from the score rows); any further ones are counted for the
+// in-kernel rescan.  One CTA.
+__global__ void rescan_plan_kernel(const int32_t* __restrict__ fail_list,
+                                   const int* __restrict__ fail_count,
+                                   const int32_t* __restrict__ qo, int S,
+                                   const int32_t* __restrict__ q_pos, int4* __restrict__ groups,
+                                   int* __restrict__ counts) {
+  pdl_wait_then_release();
+  const int n = *fail_count;
+  const int g = n < kRescanCap ? n : kRescanCap;
+  for (int i = threadIdx.x; i < g; i += blockDim.x) {
+    const int t = fail_list[i];
+    groups[i] = make_int4(upper_segment<int32_t>(qo, S, t), t, t + 1, q_pos[t]);
+  }
+  if (threadIdx.x == 0) {
+    counts[0] = g;
+    counts[1] = n - g;
+  }
 }
 
 template <int MH>
@@ -1162,13 +1250,38 @@ int launch_pair(const StreamArgs& a, const CUtensorMap& kmap, const CUtensorMap&
   } else if ((rc = launch_one<MH>(a, kmap, qmap, sc, main_ls, st))) {
     return rc;
   }
-  // Queries whose probe threshold did not verify: rescan without a probe,
-  // one query per group, with lists that hold every key.
-  Sched fx = sc;
-  fx.fail_in = a.fail_list;
-  fx.fail_out = nullptr;
-  fx.count = a.fail_count;
+  // Queries whose probe threshold did not verify are scored again without a
+  // threshold.  The first kRescanCap: their full score rows by the split
+  // decode-path scorer (several CTAs per query), then the top-k of each row.
   prof_count("#rescan_queries", a.fail_count, st);
+  int4* rgroups = reinterpret_cast<int4*>(base + cl.main_lists + cl.main_counts + cl.fix_lists +
+                                          cl.fix_counts + cl.rescan_rows);
+  int* rcounts = reinterpret_cast<int*>(rgroups + kRescanCap);  // {by rows, rest}
+  float* rrows = reinterpret_cast<float*>(base + cl.main_lists + cl.main_counts + cl.fix_lists +
+                                          cl.fix_counts);
+  {
+    ProfScope ps("rescan_plan", st);
+    rc = cuda_fail(launch_pdl(rescan_plan_kernel, dim3(1), dim3(128), 0, st,
+                              (const int32_t*)a.fail_list, (const int*)a.fail_count,
+                              a.p->query_offsets, a.p->num_seqs, a.p->q_pos, rgroups, rcounts),
+                   "rescan_plan_kernel");
+    if (rc) return rc;
+  }
+  ScoreArgs ra;
+  ra.p = a.p; ra.qsel = a.qsel; ra.wsel = a.wsel; ra.m = a.m; ra.K = a.K; ra.cand = nullptr;
+  ra.k_cand = 0; ra.groups = rgroups; ra.group_count = rcounts; ra.max_groups = kRescanCap;
+  ra.G = 1; ra.q_lo = 0; ra.I = rrows; ra.ld = cl.row_ld; ra.max_tiles = cl.rows_full;
+  ra.row_by_group = true;
+  if ((rc = launch_score(ra, st))) return rc;
+  if ((rc = launch_topk(*a.p, rrows, cl.row_ld, nullptr, 0, 0, kRescanCap, a.k, a.idx, a.val, st,
+                        a.fail_list, rcounts)))
+    return rc;
+  // Any further ones: rescan inside the streaming kernel, one query per
+  // group, with lists that hold every key.
+  Sched fx = sc;
+  fx.fail_in = a.fail_list + kRescanCap;
+  fx.fail_out = nullptr;
+  fx.count = rcounts + 1;
   return launch_one<MH>(a, kmap, qmap, fx, fix_ls, st);
 }
 
@@ -1183,7 +1296,8 @@ int64_t stream_subcap(int max_seq_len) {
 
 size_t stream_cand_bytes(int grid, int64_t subcap, int m) {
   const CandLayout c = cand_layout(grid, subcap, kN / m);
-  return c.main_lists + c.main_counts + c.fix_lists + c.fix_counts;
+  return c.main_lists + c.main_counts + c.fix_lists + c.fix_counts + c.rescan_rows +
+         c.rescan_groups;
 }
 
 size_t stream_deferred_bytes(int T, int64_t subcap, int k) {

@@ -81,13 +81,15 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     topk_kernel(const float* __restrict__ I, int64_t ld, const int32_t* __restrict__ tok,
                 int n_fixed, const int64_t* __restrict__ ko, const int32_t* __restrict__ qo,
                 const int32_t* __restrict__ q_pos, int S, int q_lo, int k,
-                int32_t* __restrict__ idx_out, float* __restrict__ val_out, uint32_t* status) {
+                int32_t* __restrict__ idx_out, float* __restrict__ val_out, uint32_t* status,
+                const int32_t* __restrict__ rows_list, const int* __restrict__ rows_count) {
   pdl_wait_then_release();
+  if (rows_list && (int)blockIdx.x >= *rows_count) return;
   __shared__ uint32_t hist[kMaxBins];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sel_bin, sel_above, sel_count, n_valid, out_cnt;
 
-  const int t = q_lo + blockIdx.x;
+  const int t = rows_list ? rows_list[blockIdx.x] : q_lo + (int)blockIdx.x;
   const int s = upper_segment<int32_t>(qo, S, t);
   const int64_t L = ko[s + 1] - ko[s];
   int pos = q_pos[t];
@@ -229,7 +231,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
                         int n_fixed, const int64_t* __restrict__ ko,
                         const int32_t* __restrict__ qo, const int32_t* __restrict__ q_pos, int S,
                         int q_lo, int k, int C, int32_t* __restrict__ idx_out,
-                        float* __restrict__ val_out, uint32_t* status) {
+                        float* __restrict__ val_out, uint32_t* status,
+                        const int32_t* __restrict__ rows_list,
+                        const int* __restrict__ rows_count) {
   pdl_wait_then_release();
   extern __shared__ __align__(16) uint64_t keys[];  // [kClusterCap]; 0 = not a candidate
   __shared__ uint32_t hist[2][kMaxBins];
@@ -239,7 +243,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
 
   const uint32_t rank = cluster_ctarank();
   const int row = blockIdx.x / C;
-  const int t = q_lo + row;
+  // (uniform over the cluster: every CTA of it has the same row)
+  if (rows_list && row >= *rows_count) return;
+  const int t = rows_list ? rows_list[row] : q_lo + row;
   const int s = upper_segment<int32_t>(qo, S, t);
   const int64_t L = ko[s + 1] - ko[s];
   int pos = q_pos[t];
@@ -393,7 +399,7 @@ int topk_cluster_size(int rows, int64_t nmax, int sms) {
 
 int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32_t* tok,
                 int n_fixed, int q_lo, int q_hi, int k, int32_t* idx, float* val,
-                cudaStream_t st) {
+                cudaStream_t st, const int32_t* rows_list, const int* rows_count) {
   if (q_hi <= q_lo) return MISA_OK;
   const int rows = q_hi - q_lo;
   const int64_t nmax = tok ? n_fixed : p.max_seq_len;
@@ -417,16 +423,16 @@ int launch_topk(const misa_problem_t& p, const float* I, int64_t ld, const int32
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    ProfScope ps("topk", st);
+    ProfScope ps(rows_list ? "rescan_topk" : "topk", st);
     cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, I, ld, tok, n_fixed,
                                        p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs, q_lo,
-                                       k, C, idx, val, status_ptr());
+                                       k, C, idx, val, status_ptr(), rows_list, rows_count);
     return cuda_fail(e, "topk_cluster_kernel");
   }
-  ProfScope ps("topk", st);
+  ProfScope ps(rows_list ? "rescan_topk" : "topk", st);
   return cuda_fail(launch_pdl(topk_kernel, dim3(q_hi - q_lo), dim3(kTopkThreads), 0, st, I, ld,
                               tok, n_fixed, p.key_offsets, p.query_offsets, p.q_pos, p.num_seqs,
-                              q_lo, k, idx, val, status_ptr()),
+                              q_lo, k, idx, val, status_ptr(), rows_list, rows_count),
                    "topk_kernel");
 }
 

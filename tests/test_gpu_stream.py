@@ -204,9 +204,10 @@ def test_stream_probe_overestimate_goes_through_fixup():
     prof = misa.profile_collect()
     misa.profile_enable(False)
     status_ok()
-    assert "score_fixup" in prof
-    # the queries with the overestimating sample (long enough to be probed)
+    # the queries with the overestimating sample (long enough to be probed):
+    # more than the split rescan takes, so both rescan paths run
     assert prof["#rescan_queries"][1] > 1000
+    assert "rescan_score" in prof and "rescan_topk" in prof and "score_fixup" in prof
     si, sv = ix.idx.clone(), ix.val.clone()
     dbg = torch.empty((wl.T, L), dtype=torch.float32, device="cuda")
     misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, Kd, wl.k, ix.idx, ix.val, ix.ws, dbg)
@@ -279,3 +280,46 @@ def test_stream_dense_rescan_at_prefill_size():
     sel = torch.tensor(rows, device="cuda")
     parity.check_dense_rows(wl, rows, ix.idx[sel].cpu().numpy(),
                             ix.val[sel].cpu().numpy()).assert_ok()
+
+
+def test_stream_few_failures_rescanned_as_score_rows():
+    # Six 1940-key sequences, k = 512: only queries with at least 16 tiles of
+    # prefix (positions 1920..1939) are probed, and the probe tile (tile 12)
+    # holds the high scores of the overestimate pattern, so about 20 queries
+    # per sequence fail: fewer than the split rescan takes (128), which
+    # scores them as full rows over several CTAs each and selects from those.
+    lens = [1940] * 6
+    H, d = 8, 128
+    wl = make_workload(seq_lens=lens, queries="all", H=H, B=64, m=8, k=512, seed=12,
+                       needles=False)
+    L = sum(lens)
+    K = np.zeros((L, d), np.float32)
+    K[:, 0] = 1.0
+    s = np.concatenate([np.arange(n) for n in lens])
+    high = ((s // 128) % 8 == 4) & (s % 2 == 0)
+    K[high, 0] = 10.0
+    K[:, 1] = (s % 5) * 0.25
+    q = np.zeros((wl.T, H, d), np.float32)
+    q[:, :, 0] = 1.0
+    q[:, :, 1] = 0.5
+    wl = dataclasses.replace(wl, K_bits=f32_to_bf16_bits(K), q_bits=f32_to_bf16_bits(q),
+                             w=np.full((wl.T, H), 0.125, np.float32))
+    prob, Kd, qd, wd = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    misa.profile_enable(True)
+    ix.misa(qd, wd, Kd)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    n_fail = prof["#rescan_queries"][1]
+    assert 0 < n_fail <= 128, n_fail
+    si, sv = ix.idx.clone(), ix.val.clone()
+    dbg = torch.empty((wl.T, max(lens)), dtype=torch.float32, device="cuda")
+    misa.score_topk(prob, ix.q_r, ix.w_r, wl.m, Kd, wl.k, ix.idx, ix.val, ix.ws, dbg)
+    status_ok()
+    same_sets(si, sv, ix.idx, ix.val)
+    invariants(wl, si)
+    rows = [1935, 1939, 1940 + 1925, 5 * 1940 + 1939]
+    sel = torch.tensor(rows, device="cuda")
+    parity.check_misa_rows(wl, rows, si[sel].cpu().numpy(), sv[sel].cpu().numpy(),
+                           heads=ix.heads[sel].cpu().numpy()).assert_ok()
