@@ -54,6 +54,9 @@ def parse():
                     help="skip the routed-heads x block-pruning comparison (decode workloads)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the --config workload (no per_config object)")
+    ap.add_argument("--shard", choices=["none", "queries"], default="none",
+                    help="queries: the N ranks split ONE problem's query rows (K replicated, "
+                         "results all-gathered; strong scaling) instead of each running its own")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--max-queries", type=int, default=0,
                     help="keep only the last N queries (small captures for ncu)")
@@ -431,11 +434,21 @@ class Bench:
         from misa_synth import CONFIGS, make_config
         self.misa, self.torch, self.np = misa, torch, np
         self.cfg, self.args, self.world, self.dev = cfg, args, world, dev
-        wl = make_config(cfg, seed=rank_seed(cfg, rank))
+        # --shard queries: every rank draws the same problem and keeps its
+        # range of query rows (sharding.query_ranges); otherwise each rank
+        # draws its own problem
+        self.shard = getattr(args, "shard", "none") == "queries" and world > 1
+        wl = make_config(cfg, seed=rank_seed(cfg, 0 if self.shard else rank))
         if args.k_cand >= 0 and cfg == args.config:
             wl = dc.replace(wl, k_cand=args.k_cand)
         if args.max_queries and args.max_queries < wl.T:
             wl = wl.subset_queries(range(wl.T - args.max_queries, wl.T))
+        self.job_pairs = wl.pairs * (1 if self.shard else world)
+        self.ranges = None
+        if self.shard:
+            from long_context_sparse_misa_b200 import sharding
+            self.ranges = sharding.query_ranges(wl.q_pos, world)
+            wl = wl.subset_queries(range(*self.ranges[rank]))
         self.wl = wl
         self.hier = bool(wl.k_cand)
         self.decode = CONFIGS[cfg]["queries"] != "all"
@@ -545,8 +558,15 @@ class Bench:
     def misa_step(self):
         ix = self.ix
         if self.hier:
-            return ix.hier(self.q, self.w, self.K, pool_from=self.pool_from)
-        return ix.misa(self.q, self.w, self.K, pool_from=self.pool_from)
+            out = ix.hier(self.q, self.w, self.K, pool_from=self.pool_from)
+        else:
+            out = ix.misa(self.q, self.w, self.K, pool_from=self.pool_from)
+        if self.shard:
+            # every rank ends the step with the whole problem's selection
+            from long_context_sparse_misa_b200 import sharding
+            self.all_idx = sharding.gather_rows(ix.idx, self.ranges)
+            self.all_val = sharding.gather_rows(ix.val, self.ranges)
+        return out
 
 
 def summarise_kernels(kerns, steps):
@@ -587,7 +607,7 @@ def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
     k = kernels.get("score", {"ms_per_step": float("nan"), "launches_per_step": 0})
     streamed = "topk" not in kernels
     res = {"workload": bn.workload, "ms_per_step": ms, "latency_ms": ms,
-           "value": job_throughput(wl.pairs, world, ms), "unit": UNIT,
+           "value": bn.job_pairs / (ms / 1e3), "unit": UNIT,
            "step_ms_p50": p50, "step_ms_p90": p90, "cuda_graph": bn.use_graph,
            "roofline": roofline_of(wl, k["ms_per_step"], k["launches_per_step"], streamed, peaks,
                                    clk, bn.workload),
@@ -606,7 +626,7 @@ def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
         d_k_ms = d_kernels.get("score", {"ms_per_step": float("nan")})["ms_per_step"]
         rec, iou = recall_iou_rows(misa_idx, ix.idx)
         res["dense_dsa"] = {
-            "ms_per_step": dms, "value": job_throughput(wl.pairs, world, dms), "unit": UNIT,
+            "ms_per_step": dms, "value": bn.job_pairs / (dms / 1e3), "unit": UNIT,
             "misa_speedup": dms / ms,
             "kernels": {n: v["ms_per_step"] for n, v in d_kernels.items()},
             "rescanned_queries_per_step": d_cnt.get("rescan_queries", 0) / dsteps}
@@ -636,7 +656,7 @@ def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
                                     bsteps, warmup=1)
         bms = max_over_ranks(sum(b_ms), world) / bsteps
         blk = {"n_blocks": nb, "candidates_per_query": (nb + 1) * wl.B,
-               "ms_per_step": bms, "value": job_throughput(wl.pairs, world, bms), "unit": UNIT,
+               "ms_per_step": bms, "value": bn.job_pairs / (bms / 1e3), "unit": UNIT,
                "speedup_vs_misa": ms / bms,
                "recall_of_misa_selection": recall_iou_rows(bx.idx, misa_idx)[0],
                "kernels": {n: v["ms_per_step"] for n, v in summarise_kernels(b_kerns, bsteps).items()}}
@@ -714,7 +734,7 @@ def e2e_leg(bn, args, world):
     pipeline(e2e_steps, e0, e1)
     torch.cuda.synchronize()
     ems = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    return {"value": job_throughput(wl.pairs, world, ems), "unit": UNIT, "ms_per_step": ems,
+    return {"value": bn.job_pairs / (ems / 1e3), "unit": UNIT, "ms_per_step": ems,
             "h2d_bytes_per_step": K_h.nbytes + q_h.nbytes + w_h.nbytes,
             "d2h_bytes_per_step": outs_h[0][0].nbytes + outs_h[0][1].nbytes,
             "pipelined": "uploads and downloads on a copy stream, double buffered"}
@@ -739,11 +759,14 @@ def run_ours(args):
     wl = bn.wl
     line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if bn.shard else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)/sqrt(d) bf16 q,k with 1% planted needles; "
                     "w ~ N(0,1)/sqrt(H) fp32)",
             "config": workload_config(wl, args.config) | {
-                "parallelism": f"independent problem per GPU x{world}"}}
+                "parallelism": (f"query shards of one problem x{world} (K replicated, idx/val "
+                                "all-gathered every step)") if bn.shard
+                               else f"independent problem per GPU x{world}"}}
     if bn.decode:
         line["config"]["decode_step"] = "pooled keys of earlier blocks kept; blocks with new keys re-pooled"
     line |= {k_: v for k_, v in res.items() if k_ not in ("value", "unit", "ms_per_step", "workload")}
