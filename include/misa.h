@@ -27,6 +27,11 @@
  *     (score desc, token index asc); -0 counts as +0.  A query whose prefix is
  *     shorter than k selects every prefix token and pads its row with index
  *     -1 and value -inf.  Row order of idx/val is unspecified.
+ *   - NaN (from a NaN in q, w or K): a head whose router score is NaN is
+ *     ranked last and MISA_STATUS_BAD_INPUT is set; a NaN token score ranks
+ *     below every number, so it is selected only when its row has fewer
+ *     other scores than min(k, prefix length), and then (with value NaN)
+ *     the same bit is set.
  */
 #ifndef MISA_H_
 #define MISA_H_
@@ -55,7 +60,8 @@ enum {
 /* Bits of the device status word. */
 #define MISA_STATUS_TIMEOUT   0x1u /* a bounded wait in a kernel gave up; that CTA returned early */
 #define MISA_STATUS_BOUNDS    0x2u /* an index fell outside its buffer; the access was skipped */
-#define MISA_STATUS_BAD_INPUT 0x4u /* a query position or candidate outside its sequence, or a NaN score */
+#define MISA_STATUS_BAD_INPUT 0x4u /* a query position or candidate outside its sequence, a NaN
+                                      router score, or a NaN token score in a selection */
 
 /*
  * Problem description (the shapes of one indexer call).

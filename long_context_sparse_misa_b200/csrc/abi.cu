@@ -665,7 +665,7 @@ int misa_stream_status(misa_stream_t stream, int32_t* device_status) {
   if (device_status) *device_status = (int32_t)v;
   if (v & MISA_STATUS_TIMEOUT) { set_error("a device wait timed out"); return MISA_ERR_DEVICE_TIMEOUT; }
   if (v & MISA_STATUS_BOUNDS) { set_error("a device index was out of range"); return MISA_ERR_DEVICE_BOUNDS; }
-  if (v & MISA_STATUS_BAD_INPUT) { set_error("bad input (position, candidate or NaN)"); return MISA_ERR_DEVICE_BAD_INPUT; }
+  if (v & MISA_STATUS_BAD_INPUT) { set_error("bad input (position, candidate or a NaN score)"); return MISA_ERR_DEVICE_BAD_INPUT; }
   return MISA_OK;
 }
 

@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kBlkPerCta)
   }
   float score = 0.f;
 #pragma unroll
-  for (int j = 0; j < M; ++j) score = fmaf(ws[j], fmaxf(acc[j], 0.f), score);
+  for (int j = 0; j < M; ++j) score = fmaf(ws[j], relu_nan(acc[j]), score);
   Sb[o] = score;
   btok[o] = b;
 }

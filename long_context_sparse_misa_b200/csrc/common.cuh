@@ -330,6 +330,15 @@ __device__ __forceinline__ float sum_pair(uint64_t acc) {
   return a0 + a1;
 }
 
+// ReLU that keeps a NaN (max.NaN): as in the oracle's arithmetic, a NaN in
+// q, w or a key reaches the score it feeds (fmaxf would drop it for 0), so a
+// NaN router score can be flagged and ranked last.
+__device__ __forceinline__ float relu_nan(float x) {
+  float r;
+  asm("max.NaN.f32 %0, %1, 0f00000000;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Head-weighted ReLU sum of one query's MH accumulator columns, the one
 // summation order every scoring kernel uses (so all paths agree bit for bit):
 // even heads into a0, odd heads into a1 (one packed FMA per pair), then

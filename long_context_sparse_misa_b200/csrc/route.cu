@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           ffma2(d2, d3, qreg[4 * i + 6], qreg[4 * i + 7], c.z, c.w);
           ffma2(e2, e3, qreg[4 * i + 6], qreg[4 * i + 7], c1.z, c1.w);
         }
-        acc += fmaxf((d0 + d1) + (d2 + d3), 0.f);
-        acc += fmaxf((e0 + e1) + (e2 + e3), 0.f);
+        acc += relu_nan((d0 + d1) + (d2 + d3));
+        acc += relu_nan((e0 + e1) + (e2 + e3));
       }
       for (; b < lim; ++b) {
         const float4* row = reinterpret_cast<const float4*>(kb + b * kD);
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           ffma2(d2, d3, qreg[4 * i + 4], qreg[4 * i + 5], c.x, c.y);
           ffma2(d2, d3, qreg[4 * i + 6], qreg[4 * i + 7], c.z, c.w);
         }
-        acc += fmaxf((d0 + d1) + (d2 + d3), 0.f);
+        acc += relu_nan((d0 + d1) + (d2 + d3));
       }
     }
   }
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         d = fmaf(qreg[4 * i + 2], a.z, d);
         d = fmaf(qreg[4 * i + 3], a.w, d);
       }
-      acc += fmaxf(d, 0.f);
+      acc += relu_nan(d);
     }
   }
 
@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(kMmaBlock, 1)
           float c[4];
           mma_rows(c, afr, khi, klo, nt * 8);
           const int b0 = c0 + nt * 8 + 2 * ti;  // blocks of columns 2ti, 2ti + 1
-          accA += (b0 < fA ? fmaxf(c[0], 0.f) : 0.f) + (b0 + 1 < fA ? fmaxf(c[1], 0.f) : 0.f);
-          accB += (b0 < fB ? fmaxf(c[2], 0.f) : 0.f) + (b0 + 1 < fB ? fmaxf(c[3], 0.f) : 0.f);
+          accA += (b0 < fA ? relu_nan(c[0]) : 0.f) + (b0 + 1 < fA ? relu_nan(c[1]) : 0.f);
+          accB += (b0 < fB ? relu_nan(c[2]) : 0.f) + (b0 + 1 < fB ? relu_nan(c[3]) : 0.f);
         }
       }
     }
@@ -469,10 +469,10 @@ __global__ void __launch_bounds__(kMmaBlock, 1)
         mma_rows(c, afr, phi, plo, nt * 8);
         const int col0 = nt * 8 + 2 * ti;
         const bool pa = qA >= 0 && fA * B != nA, pb = qB >= 0 && fB * B != nB;
-        if (pa && qA == col0) accA += fmaxf(c[0], 0.f);
-        if (pa && qA == col0 + 1) accA += fmaxf(c[1], 0.f);
-        if (pb && qB == col0) accB += fmaxf(c[2], 0.f);
-        if (pb && qB == col0 + 1) accB += fmaxf(c[3], 0.f);
+        if (pa && qA == col0) accA += relu_nan(c[0]);
+        if (pa && qA == col0 + 1) accA += relu_nan(c[1]);
+        if (pb && qB == col0) accB += relu_nan(c[2]);
+        if (pb && qB == col0 + 1) accB += relu_nan(c[3]);
       }
     }
   }

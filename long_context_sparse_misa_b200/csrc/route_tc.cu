@@ -348,8 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int x = 0; x < 32; x += 2) {
-                a0 += fmaxf(v[j][x], 0.f);
-                a1 += fmaxf(v[j][x + 1], 0.f);
+                a0 += relu_nan(v[j][x]);
+                a1 += relu_nan(v[j][x + 1]);
               }
             acc[sub] += a0 + a1;
           } else if (nvis > 0) {
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int x = 0; x < 32; ++x)
-                if (j * 32 + x < nvis) a0 += fmaxf(v[j][x], 0.f);
+                if (j * 32 + x < nvis) a0 += relu_nan(v[j][x]);
             acc[sub] += a0;
           }
         }
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dp = fmaf(__uint_as_float(u.w << 16), Pq[8 * i + 6], dp);
               dp = fmaf(__uint_as_float(u.w & 0xFFFF0000u), Pq[8 * i + 7], dp);
             }
-            total += fmaxf(dp, 0.f);
+            total += relu_nan(dp);
           }
           r = __ldg(w + (int64_t)(qb + qi) * H + h) * total;
           if (router_scores) router_scores[(int64_t)(qb + qi) * H + h] = r;

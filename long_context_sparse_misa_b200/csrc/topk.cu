@@ -167,6 +167,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
       if (slot < (uint32_t)k) {
         idx[slot] = token;
         val[slot] = v + 0.0f;
+        // NaN ranks below every number, so it is selected only to fill a row
+        // that has fewer numbers than the row needs
+        if (v != v) set_status(status, MISA_STATUS_BAD_INPUT);
       } else {
         set_status(status, MISA_STATUS_BOUNDS);  // duplicate tokens in a candidate row
       }
@@ -367,6 +370,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     if (slot < (uint32_t)k) {
       idx[slot] = (int)(0xFFFFFFFFu - (uint32_t)key);
       val[slot] = key_to_float((uint32_t)(key >> 32));
+      if ((uint32_t)(key >> 32) == 0u) set_status(status, MISA_STATUS_BAD_INPUT);  // a NaN
     } else {
       set_status(status, MISA_STATUS_BOUNDS);  // duplicate tokens in a candidate row
     }

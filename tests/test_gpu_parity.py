@@ -317,3 +317,50 @@ def test_config_prefill_dense_sampled_rows(cfg):
           f"rescanned queries={rescans}")
     # the sampled threshold holds for all but a few queries
     assert rescans <= wl.T // 100
+
+
+# ------------------------------------------------------------------ NaN inputs
+NAN_BF16 = np.uint16(0x7FC0)
+
+
+def test_nan_router_score_ranks_the_head_last_and_is_flagged():
+    wl = ragged(seed=51, H=16, m=4, k=60)
+    wl.q_bits[3, 5, 17] = NAN_BF16          # one element of head 5 of query row 3
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=4, k=60)
+    ix.misa(q, w, K)
+    code, bits = misa.stream_status()
+    assert bits & 0x4 and code == 7
+    heads = ix.heads.cpu().numpy()
+    assert 5 not in heads[3].tolist()
+    # every row (the NaN head left out of row 3) against the oracle, whose
+    # router also ranks the NaN score last
+    parity.check_misa_rows(wl, range(wl.T), ix.idx.cpu().numpy(), ix.val.cpu().numpy(),
+                           heads=heads, m=4).assert_ok()
+    status_ok()
+
+
+@pytest.mark.parametrize("streamed", [False, True])
+def test_nan_token_scores_fill_only_short_rows_and_are_flagged(streamed):
+    if streamed:
+        wl = make_workload(seq_lens=[10000], queries="all", H=8, B=64, m=8, k=64, seed=52)
+        bad = 7000
+    else:
+        wl = ragged(seed=52, H=8, m=8, k=60)
+        bad = 9                               # position 128 of the first sequence
+    wl.w[bad, :] = np.nan                     # every head of one query: all its scores NaN
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=8, k=wl.k)
+    ix.dense(q, w, K)
+    code, bits = misa.stream_status()
+    assert bits & 0x4 and code == 7
+    idx, val = ix.idx.cpu().numpy(), ix.val.cpu().numpy()
+    n = int(wl.q_pos[bad]) + 1
+    kk = min(wl.k, n)
+    # no numbers in the row: the first min(k, n) tokens (ties go to the lower index), value NaN
+    assert sorted(idx[bad][idx[bad] >= 0].tolist()) == list(range(kk))
+    assert np.isnan(val[bad][:kk]).all() if not streamed else np.isnan(val[bad][idx[bad] >= 0]).all()
+    rows = [i for i in (list(range(wl.T)) if not streamed else [0, 2047, 5000, 6999, 7001, 9999])
+            if i != bad]
+    parity.check_dense_rows(wl, rows, idx[rows], val[rows]).assert_ok()
+    status_ok()
