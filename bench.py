@@ -88,9 +88,10 @@ def score_src_sha(kernel: str = "score_stream"):
     return h.hexdigest()[:16]
 
 
-def traffic_per_pair(kernel: str, workload: str):
-    """DRAM bytes per scored pair from a committed ncu summary whose kernel
-    source hash matches the current source; None otherwise."""
+def profile_traffic(kernel: str, workload: str):
+    """DRAM traffic of one kernel from a committed ncu summary whose kernel
+    source hash matches the current source: ("pair", bytes per scored pair)
+    or ("query", bytes per query row); None when no summary matches."""
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
@@ -103,10 +104,10 @@ def traffic_per_pair(kernel: str, workload: str):
         m_k = re.search(r"^kernel:\s*(\S+)", text, re.M)
         m_w = re.search(r"^workload:\s*(\S+)", text, re.M)
         m_s = re.search(r"^source_sha:\s*(\S+)", text, re.M)
-        m_t = re.search(r"^dram_bytes_per_pair:\s*([0-9.eE+-]+)", text, re.M)
+        m_t = re.search(r"^dram_bytes_per_(pair|query):\s*([0-9.eE+-]+)", text, re.M)
         if m_k and m_w and m_s and m_t and m_k.group(1) == kernel and \
                 m_w.group(1) == workload and m_s.group(1) == sha:
-            return float(m_t.group(1))
+            return m_t.group(1), float(m_t.group(2))
     return None
 
 
@@ -392,7 +393,7 @@ def roofline_of(wl, prof_ms, launches_per_step, streamed, peaks, clk, workload):
     """Roofline of the dominant kernel (routed scoring) from its CUDA-event
     time per step."""
     pairs = wl.pairs
-    tpp = traffic_per_pair("score_stream" if streamed else "score", workload)
+    tp = profile_traffic("score_stream" if streamed else "score", workload)
     sec = prof_ms / 1e3
     if streamed:
         # prefill: a dense contraction, 2*m*d flops per scored pair.  The
@@ -416,7 +417,8 @@ def roofline_of(wl, prof_ms, launches_per_step, streamed, peaks, clk, workload):
              "algorithmic_bytes_per_launch": abytes / max(launches_per_step, 1)}
     r |= {"launches_per_step": launches_per_step, "kernel_ms_per_step": prof_ms,
           "sm_mhz_median": clk.get("sm_mhz"),
-          "traffic": None if tpp is None else tpp * pairs / max(launches_per_step, 1)}
+          "traffic": None if tp is None else
+              tp[1] * (pairs if tp[0] == "pair" else wl.T) / max(launches_per_step, 1)}
     return r
 
 

@@ -72,12 +72,16 @@ def test_profile_traffic_lookup_matches_kernel_workload_and_source_hash(tmp_path
     (tmp_path / "profiles" / "b.md").write_text(
         "# y\n\nkernel: score_stream\nworkload: w2\nsource_sha: 0000000000000000\n"
         "dram_bytes_per_pair: 9.0\n")
+    (tmp_path / "profiles" / "c.md").write_text(
+        f"# z\n\nkernel: score_stream\nworkload: w4\nsource_sha: {sha}\n"
+        "dram_bytes_per_query: 93800\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "score_src_sha", lambda kernel="score_stream": sha)
-    assert bench.traffic_per_pair("score_stream", "w1") == 1.5
-    assert bench.traffic_per_pair("score_stream", "w2") is None     # stale hash
-    assert bench.traffic_per_pair("score", "w1") is None            # other kernel
-    assert bench.traffic_per_pair("score_stream", "w3") is None     # no summary
+    assert bench.profile_traffic("score_stream", "w1") == ("pair", 1.5)
+    assert bench.profile_traffic("score_stream", "w2") is None     # stale hash
+    assert bench.profile_traffic("score", "w1") is None            # other kernel
+    assert bench.profile_traffic("score_stream", "w3") is None     # no summary
+    assert bench.profile_traffic("score_stream", "w4") == ("query", 93800.0)
 
 
 def test_source_hash_depends_on_the_kernel():
