@@ -21,8 +21,12 @@
 // are added in shared memory); an accumulator is released as soon as both
 // halves are copied to registers.  The causal partial block
 // of every key position (the running mean of its block up to that key) is
-// computed beforehand by one warp per pooled block, so each query only
-// reads its row.  Persistent: one CTA per SM walks its groups; the next
+// computed beforehand by one warp per pooled block; the epilogue stages the
+// group's rows of it (again as a bf16 hi + lo pair, 128-byte swizzle) and
+// the MMA warp runs one more round of N = 16 columns, column j = query j's
+// partial block, so that each (query, head) row's partial-block affinity is
+// the accumulator element in its own query's column.  Persistent: one CTA
+// per SM walks its groups; the next
 // group's q rows load as soon as the current group's MMAs are done, and its
 // MMAs start while the epilogue still ranks the current group's heads.
 #include "common.cuh"
@@ -42,16 +46,17 @@ constexpr int kHalfBytes = kStageBytes / 2;
 constexpr int kQHalfBytes = kRows * 128;              // 64 KB per 64-dim half
 constexpr int kQBytes = 2 * kQHalfBytes;
 constexpr int kMaxG = 16;                             // queries per group
-constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kRows * 4 /*r*/ +
-                           2 * kRows * 4 /*racc*/ + kMaxG * kD * 4 /*pm*/ + kMaxG * 4 * 2 +
-                           16 * 8 + 16;
+constexpr int kPmHalfBytes = kMaxG * 128;             // partial-block rows, one 64-dim half
+constexpr int kPmBytes = 2 * 2 * kPmHalfBytes;        // hi and lo, two halves each
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kPmBytes + kRows * 4 /*r*/ +
+                           2 * kRows * 4 /*racc*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
 
 struct Smem {
   uint8_t* q;
   uint8_t* k;
-  float* r;     // [kRows] router scores of the group
+  uint8_t* pm;  // [hi, lo][2 halves][kMaxG rows][128 B]: running block means at the queries
+  float* r;     // [kRows] partial-block affinity, then router score, of each row
   float* racc;  // [2][kRows] block-axis ReLU sums of each half of the chunks
-  float* pm;    // [kMaxG][128] running block means at the group's query positions
   int* pos;
   int* flags;
   uint64_t* full;
@@ -60,6 +65,7 @@ struct Smem {
   uint64_t* tempty;  // [4]
   uint64_t* qfull;
   uint64_t* qempty;
+  uint64_t* pmfull;
   uint64_t* drain;
   uint32_t* tmem_slot;
   int* abort;
@@ -71,10 +77,10 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.q = p;
   s.k = p + kQBytes;
-  s.r = reinterpret_cast<float*>(s.k + kStages * kStageBytes);
+  s.pm = s.k + kStages * kStageBytes;  // 1024-byte aligned
+  s.r = reinterpret_cast<float*>(s.pm + kPmBytes);
   s.racc = s.r + kRows;
-  s.pm = s.racc + 2 * kRows;
-  s.pos = reinterpret_cast<int*>(s.pm + kMaxG * kD);
+  s.pos = reinterpret_cast<int*>(s.racc + 2 * kRows);
   s.flags = s.pos + kMaxG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
   s.full = bars;
@@ -83,7 +89,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tempty = s.tfull + 1;
   s.qfull = s.tempty + 4;
   s.qempty = s.qfull + 1;
-  s.drain = s.qempty + 1;
+  s.pmfull = s.qempty + 1;
+  s.drain = s.pmfull + 1;
   s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_slot + 1);
   return s;
@@ -171,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) mbar_init(&s.tempty[i], kEpiWarps);
     mbar_init(s.qfull, 1);
     mbar_init(s.qempty, 1);
+    mbar_init(s.pmfull, kEpiWarps);
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
@@ -263,6 +271,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) umma_commit(s.tfull);
         }
+        // Partial blocks: N = 16 columns (query j's running block mean, hi
+        // then lo) into the first columns of every accumulator.
+        if (ok && (ok = mbar_wait(s.pmfull, gl & 1, s.abort, status))) {
+          tc_fence_after();
+          const uint32_t pm_addr = smem_u32(s.pm);
+          const uint32_t idesc16 = idesc_bf16_f32(128, kMaxG);
+#pragma unroll
+          for (int sub = 0; sub < NSUB; ++sub) {
+            if (!(ok = mbar_wait(&s.tempty[sub], (cc & 1) ^ 1, s.abort, status))) break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + sub * kChunk;
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+              for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t a = sw128_kmajor_desc(q_addr + (kk >> 2) * kQHalfBytes +
+                                                     sub * 128 * 128 + off);
+                const uint64_t b = sw128_kmajor_desc(pm_addr + part * 2 * kPmHalfBytes +
+                                                     (kk >> 2) * kPmHalfBytes + off);
+                umma_bf16(d, a, b, idesc16, (part > 0 || kk > 0) ? 1u : 0u);
+              }
+          }
+          if (ok) umma_commit(s.tfull);
+          ++cc;
+        }
         umma_commit(s.qempty);  // q rows free once this group's MMAs are done
         ++gl;
       }
@@ -304,15 +338,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         s.pos[et] = p;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-      // The queries' running block means (partial block), staged for the
-      // head rows of each query (coalesced 16-byte loads).
-      for (int i = et; i < nq * (kD / 4); i += kEpiThreads) {
-        const int qi = i / (kD / 4), c4 = i - qi * (kD / 4);
-        const int p = s.pos[qi];
-        if (p >= 0 && (p + 1) % B != 0)
-          reinterpret_cast<float4*>(s.pm + qi * kD)[c4] =
-              __ldg(reinterpret_cast<const float4*>(Pm + (ko[seq] + p) * kD) + c4);
+      // The queries' running block means (partial block) as the B operand of
+      // the partial round: row j = query j, a bf16 hi + lo pair of the fp32
+      // mean, 128-byte swizzle (16-byte chunk c of row j at chunk c ^ (j & 7));
+      // zero rows for queries without a partial block.  One thread per
+      // (row, 8 dims).
+      for (int i = et; i < kMaxG * (kD / 8); i += kEpiThreads) {
+        const int j = i / (kD / 8), c = i - j * (kD / 8), half = c >> 3, c8 = c & 7;
+        const int p = s.pos[j];
+        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+        if (p >= 0 && (p + 1) % B != 0) {
+          const float4* src = reinterpret_cast<const float4*>(Pm + (ko[seq] + p) * kD) + 2 * c;
+          x0 = __ldg(src);
+          x1 = __ldg(src + 1);
+        }
+        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]);
+          const __nv_bfloat16 h1 = __float2bfloat16_rn(x[2 * e + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * e] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * e + 1] - __bfloat162float(h1));
+          hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const int off = half * kPmHalfBytes + j * 128 + ((c8 ^ (j & 7)) << 4);
+        *reinterpret_cast<uint4*>(s.pm + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(s.pm + 2 * kPmHalfBytes + off) =
+            make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
+      fence_proxy_async_smem();  // visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s.pmfull);
 
       // Block-axis ReLU sums: this thread owns row sub*128 + quarter*32 + lane
       // of every accumulator, columns ch*64 .. ch*64+63 of each chunk.
@@ -364,12 +422,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
+      // Partial round: row (query qi, head h) takes column qi.
+      if (!(ok = warp_wait(s.tfull, cc & 1, s.abort, status))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < NSUB; ++sub) {
+        float v[16];
+        if (ch == 0) {
+          tmem_ld16(lane_addr + sub * kChunk, v);
+          tmem_wait_ld();
+          reg_fence16(v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.tempty[sub]);
+        const int row = sub * 128 + quarter * 32 + lane;
+        if (ch == 0 && row < ROWS) {
+          const int qi = row / H;
+          float dp = 0.f;
+#pragma unroll
+          for (int j = 0; j < kMaxG; ++j) dp = j == qi ? v[j] : dp;
+          s.r[row] = dp;
+        }
+      }
+      ++cc;
 #pragma unroll
       for (int sub = 0; sub < NSUB; ++sub) {
         const int row = sub * 128 + quarter * 32 + lane;
         if (row < ROWS) s.racc[ch * kRows + row] = acc[sub];
       }
-      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");  // s.pm, s.racc complete
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");  // s.r (partial), s.racc complete
 
       for (int row = et; row < ROWS; row += kEpiThreads) {
         const int qi = row / H, h = row - qi * H;
@@ -377,24 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qi < nq && s.pos[qi] >= 0) {
           const int p = s.pos[qi];
           float total = s.racc[row] + s.racc[kRows + row];
-          if ((p + 1) % B != 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)(qb + qi) * H + h) * kD);
-            const float* Pq = s.pm + qi * kD;  // running block mean at p
-            float dp = 0.f;
-#pragma unroll
-            for (int i = 0; i < kD / 8; ++i) {
-              const uint4 u = __ldg(src + i);
-              dp = fmaf(__uint_as_float(u.x << 16), Pq[8 * i + 0], dp);
-              dp = fmaf(__uint_as_float(u.x & 0xFFFF0000u), Pq[8 * i + 1], dp);
-              dp = fmaf(__uint_as_float(u.y << 16), Pq[8 * i + 2], dp);
-              dp = fmaf(__uint_as_float(u.y & 0xFFFF0000u), Pq[8 * i + 3], dp);
-              dp = fmaf(__uint_as_float(u.z << 16), Pq[8 * i + 4], dp);
-              dp = fmaf(__uint_as_float(u.z & 0xFFFF0000u), Pq[8 * i + 5], dp);
-              dp = fmaf(__uint_as_float(u.w << 16), Pq[8 * i + 6], dp);
-              dp = fmaf(__uint_as_float(u.w & 0xFFFF0000u), Pq[8 * i + 7], dp);
-            }
-            total += relu_nan(dp);
-          }
+          if ((p + 1) % B != 0) total += relu_nan(s.r[row]);  // partial block
           r = __ldg(w + (int64_t)(qb + qi) * H + h) * total;
           if (router_scores) router_scores[(int64_t)(qb + qi) * H + h] = r;
           if (r != r) {
