@@ -139,6 +139,41 @@ def test_dense_ragged(H, k):
     parity.check_dense_rows(wl, range(wl.T), ix.idx.cpu().numpy(), ix.val.cpu().numpy()).assert_ok()
 
 
+def test_empty_sequence_between_others():
+    # A sequence with no keys (and so no queries) between two others: its
+    # zero blocks and zero rows change nothing for its neighbours.
+    wl = make_workload(seq_lens=[500, 0, 300], queries=[[10, 63, 64, 499], [], [0, 127, 299]],
+                       H=16, B=64, m=4, k=32, seed=3)
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    ix.misa(q, w, K)
+    status_ok()
+    parity.check_misa_rows(wl, range(wl.T), ix.idx.cpu().numpy(), ix.val.cpu().numpy(),
+                           heads=ix.heads.cpu().numpy(), Kbar=ix.Kbar.cpu().numpy()).assert_ok()
+    ix.dense(q, w, K)
+    status_ok()
+    parity.check_dense_rows(wl, range(wl.T), ix.idx.cpu().numpy(), ix.val.cpu().numpy()).assert_ok()
+
+
+def test_no_queries_is_a_no_op():
+    # T = 0: routing, scoring and the dense indexer return at once; only the
+    # pooling of the keys (which does not depend on the queries) runs.
+    wl = make_workload(seq_lens=[300], queries=[[]], H=8, B=16, m=2, k=4, seed=1)
+    assert wl.T == 0
+    prob, K, q, w = dev(wl)
+    ix = misa.Indexer(prob, m=wl.m, k=wl.k)
+    misa.profile_enable(True)
+    ix.misa(q, w, K)
+    ix.dense(q, w, K)
+    prof = misa.profile_collect()
+    misa.profile_enable(False)
+    status_ok()
+    assert set(prof) <= {"pool_keys"}, prof
+    assert ix.idx.shape == (0, wl.k)
+    Kbar_o = oracle.pool_keys(oracle.widen_bf16(wl.K_bits), wl.key_offsets, wl.B)
+    np.testing.assert_array_equal(ix.Kbar.cpu().numpy(), Kbar_o.astype(np.float32))
+
+
 def test_hier_whole_prefix_is_dense():
     wl = ragged(seed=31, H=64, m=8, k=40, k_cand=1024)
     prob, K, q, w = dev(wl)
