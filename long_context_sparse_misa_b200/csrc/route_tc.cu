@@ -51,7 +51,7 @@ constexpr int kMaxG = 16;                             // queries per group
 constexpr int kPmHalfBytes = kMaxG * 128;             // partial-block rows, one 64-dim half
 constexpr int kPmBytes = 2 * 2 * kPmHalfBytes;        // hi and lo, two halves each
 constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kPmBytes + kRows * 4 /*r*/ +
-                           2 * kRows * 4 /*racc*/ + kMaxG * 4 * 2 + 16 * 8 + 16;
+                           2 * kRows * 4 /*racc*/ + kMaxG * 4 /*pos*/ + 16 * 8 + 16;
 
 struct Smem {
   uint8_t* q;
@@ -59,8 +59,7 @@ struct Smem {
   uint8_t* pm;  // [hi, lo][2 halves][kMaxG rows][128 B]: running block means at the queries
   float* r;     // [kRows] partial-block affinity, then router score, of each row
   float* racc;  // [2][kRows] block-axis ReLU sums of each half of the chunks
-  int* pos;
-  int* flags;
+  int* pos;     // [kMaxG] query positions of the group (-1: none)
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -83,8 +82,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.r = reinterpret_cast<float*>(s.pm + kPmBytes);
   s.racc = s.r + kRows;
   s.pos = reinterpret_cast<int*>(s.racc + 2 * kRows);
-  s.flags = s.pos + kMaxG;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.flags + kMaxG);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.pos + kMaxG);  // 8-byte aligned
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
