@@ -607,7 +607,9 @@ def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
     p90 = max_over_ranks(step_ms[min(len(step_ms) - 1, (9 * len(step_ms)) // 10)], world)
     kernels = summarise_kernels(kerns, steps)
     k = kernels.get("score", {"ms_per_step": float("nan"), "launches_per_step": 0})
-    streamed = "topk" not in kernels
+    # the streaming prefill pass: its candidates are selected by the pass
+    # after it ("select"); decode scores rows and takes the row top-k
+    streamed = "select" in kernels
     res = {"workload": bn.workload, "ms_per_step": ms, "latency_ms": ms,
            "value": bn.job_pairs / (ms / 1e3), "unit": UNIT,
            "step_ms_p50": p50, "step_ms_p90": p90, "cuda_graph": bn.use_graph,

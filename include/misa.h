@@ -96,8 +96,9 @@ typedef struct {
  * (0 if unused), on its fastest path.  Returns 0 on invalid arguments.
  * For a prefill that streams (misa_score_topk, dsa_index_dense) this
  * includes candidate lists per query row for the exact selection after the
- * scoring pass, about T * (2 * 1.4 * k / 128 + 16) KB (8.1 GB for 131072
- * queries at k = 2048); a smaller workspace takes slower paths (selection
+ * scoring pass, about T * (2 * 1.4 * k / 128 + 16) KB with that row count
+ * between 32 and 256 (8.1 GB for 131072 queries at k = 2048, 25 GB at the
+ * MISA-dagger keep k = 8192); a smaller workspace takes slower paths (selection
  * inside the scoring kernel, then score rows with a separate top-k) and
  * MISA_ERR_WORKSPACE_TOO_SMALL only below what the slowest path needs. */
 size_t misa_workspace_size(const misa_problem_t* p, int32_t m, int32_t k, int32_t k_cand);

@@ -1132,11 +1132,16 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm)
 }
 
 // Rows of a deferred list: twice the expected candidates per lane (about
-// 1.4 k / 128 with the probe threshold) plus 16, within [32, 128] and no more
-// than one row per tile; a fuller list sends its query to the rescan.
+// 1.4 k / 128 with the probe threshold) plus 16, within [32, 256] and no more
+// than one row per tile; a fuller list sends its query to the rescan.  (The
+// selection reads a list's expected rows in any case, so a large k - the
+// MISA-dagger keep of k' = 8192, ~93 rows per lane - takes lists up to 196
+// rows rather than send every query whose busiest lane passes 128 rows, 1% at
+// 128K, to the far slower one-query rescan.)
+constexpr int kDeferredRowsCap = 256;
 int deferred_rows(int k, int64_t rows_full) {
   int64_t r = 2 * ((14 * (int64_t)k + 1279) / 1280) + 16;
-  r = r < 32 ? 32 : (r > kRowsCap ? kRowsCap : r);
+  r = r < 32 ? 32 : (r > kDeferredRowsCap ? kDeferredRowsCap : r);
   return (int)(r < rows_full ? r : rows_full);
 }
 
