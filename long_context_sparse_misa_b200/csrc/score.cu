@@ -19,8 +19,8 @@
 // head weight, and a causal compare -- no shuffles and no [m x L] tensor.
 //
 // Roles: warp 0 producer, warp 1 TMEM owner + MMA issuer (one thread),
-// warps 2..5 epilogue (TMEM lane quarter = warp % 4); in gather mode warps 6
-// and 7 are two more producers.
+// warps 2..5 epilogue (TMEM lane quarter = warp % 4); in gather mode warps 6,
+// 7 and 8 are three more producers.
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,10 +28,11 @@ namespace misa {
 namespace {
 
 constexpr int kThreads = 192;
-// Gather mode adds two producer warps (6 and 7): the copies of a tile are
-// issued by one warp, tiles go round-robin over the three producers.
-constexpr int kGatherThreads = 256;
-constexpr int kGatherProducers = 3;
+// Gather mode adds three producer warps (6, 7 and 8): the copies of a tile
+// are issued by one warp, tiles go round-robin over the four producers, one
+// per stage.
+constexpr int kGatherThreads = 288;
+constexpr int kGatherProducers = 4;
 __host__ __device__ constexpr int threads_for(bool gather) {
   return gather ? kGatherThreads : kThreads;
 }
@@ -219,8 +220,9 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
       }
     } else {
       // Gather mode: rows K[key_base + cand[t, slot]] for the 128 slots of a
-      // tile; each lane copies 4 rows as 16-byte chunks into the swizzled
-      // layout.  Producer p (warp 0, 6, 7) takes tiles p, p + 3, ...
+      // tile, copied as 16-byte chunks into the swizzled layout, two whole
+      // rows per warp instruction.  Producer p (warp 0, 6, 7, 8) takes tiles
+      // p, p + 4, ...
       const int t = qb;
       const int pos = s.pos[0];
       const int prod = warp == 0 ? 0 : warp - 5;
@@ -234,30 +236,48 @@ __global__ void __launch_bounds__(threads_for(GATHER), 1)
       }
       __syncwarp();
       // Each producer has one tile in flight: copy, wait for its copies,
-      // signal; the three producers overlap.
+      // signal; the producers overlap.  A tile's candidate indices are
+      // loaded one tile ahead, so their latency overlaps the previous
+      // tile's copies.
+      auto tile_tokens = [&](int i, int (&tk)[4]) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int slot = (tile0 + i) * kTileKeys + lane * 4 + rr;
+          tk[rr] = (i < nt && slot < k_cand) ? cand[(int64_t)t * k_cand + slot] : -1;
+        }
+      };
+      int tok_cur[4];
+      tile_tokens(prod, tok_cur);
       for (int i = prod; i < nt; i += kGatherProducers) {
         const int st = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
+        int tok_next[4];
+        tile_tokens(i + kGatherProducers, tok_next);
         if (!warp_wait(&s.empty[st], ph ^ 1, s.abort, status)) break;
         uint8_t* dst = s.k + st * kStageBytes;
+        // Two rows per copy instruction: lanes 0-15 take the 16 chunks of one
+        // row, lanes 16-31 those of the next, so each instruction reads two
+        // whole 256-byte rows (row r's token is held by lane r / 4, slot r % 4).
+        const int c = lane & 15, half = c >> 3, cc = c & 7;
+#pragma unroll 2
+        for (int u = 0; u < kTileKeys / 4; ++u) {  // rows 4u .. 4u+3, held by lane u
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = lane * 4 + rr;
-          const int slot = (tile0 + i) * kTileKeys + r;
-          int tok = slot < k_cand ? cand[(int64_t)t * k_cand + slot] : -1;
-          const bool ok = tok >= 0 && tok <= pos && key_base + tok < total_keys;
-          const uint16_t* src = K + (ok ? (key_base + tok) : 0) * kD;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int half = c >> 3, cc = c & 7;
-            cp_async_16(dst + half * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4), src + c * 8,
-                        ok);
+          for (int v = 0; v < 2; ++v) {
+            const int tA = __shfl_sync(0xffffffffu, tok_cur[2 * v], u);
+            const int tB = __shfl_sync(0xffffffffu, tok_cur[2 * v + 1], u);
+            const int r = 4 * u + 2 * v + (lane >> 4);
+            const int tok = (lane >> 4) ? tB : tA;
+            const bool ok = tok >= 0 && tok <= pos && key_base + tok < total_keys;
+            const uint16_t* src = K + (ok ? (key_base + tok) : 0) * kD + c * 8;
+            cp_async_16(dst + half * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4), src, ok);
           }
         }
         cp_async_commit();
         cp_async_wait_group<0>();
         fence_proxy_async_smem();
         mbar_arrive(&s.full[st]);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) tok_cur[rr] = tok_next[rr];
       }
       cp_async_wait_group<0>();
     }
