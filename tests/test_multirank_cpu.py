@@ -62,7 +62,7 @@ def test_single_rank_needs_no_process_group():
     assert bench.rank_seed(3, 0) == 1003
 
 
-def _shard_rank(rank, world, port, out):
+def _shard_rank(rank, world, port, out, seq_lens=(300, 1, 257), group=8):
     """One rank of a query-sharded indexer job, with the CPU oracle standing
     in for the per-rank compute: its range of query rows, then the gather."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
@@ -77,8 +77,8 @@ def _shard_rank(rank, world, port, out):
     from long_context_sparse_misa_b200 import sharding
     from misa_synth import make_workload
     bench.dist_init("gloo")
-    wl = make_workload(seq_lens=[300, 1, 257], queries="all", H=8, B=16, m=4, k=20, seed=77)
-    ranges = sharding.query_ranges(wl.q_pos, world, group=8)
+    wl = make_workload(seq_lens=list(seq_lens), queries="all", H=8, B=16, m=4, k=20, seed=77)
+    ranges = sharding.query_ranges(wl.q_pos, world, group=group)
     lo, hi = ranges[rank]
     # the shard's problem description is the workload's row subset
     sl, qo, qp = sharding.shard_metadata(wl.seq_lens, wl.query_offsets, wl.q_pos, lo, hi)
@@ -112,6 +112,24 @@ def test_query_sharded_oracle_gathers_to_the_unsharded_result():
         assert p.exitcode == 0
     assert all(ok for _, _, ok in res)
     assert sum(n for _, n, _ in res) == 558 and all(n > 0 for _, n, _ in res)
+
+
+def test_query_sharded_oracle_with_an_empty_rank():
+    # 27 queries over three ranks in 8-row groups: ranges [0,16) [16,16) [16,27),
+    # so rank 1 holds no query and rank 2 spans a sequence boundary; the padded
+    # all_gather still gives every rank the unsharded result.
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_rank, args=(r, 3, port, q, (24, 3), 8)) for r in range(3)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, _, ok in res)
+    assert [n for _, n, _ in res] == [16, 0, 11]
 
 
 def test_query_ranges_balance_causal_work():
