@@ -380,6 +380,8 @@ __device__ void final_select(uint2* region, const int* cnt, Anchor anc, int k, i
   } else {
     constexpr int kR = 4;  // rows per batch: 16 loads in flight per lane
     // Pass 0: histogram of the entries (bins relative to the query's anchor).
+    // Its loads keep the default L2 policy, so that pass 1's re-read of the
+    // same rows mostly hits L2; pass 1's are marked evict-first (last use).
     for (int i = lane; i < kBins; i += 32) selh[i] = 0u;
     __syncwarp();
     for (int r0 = 0; r0 < rows; r0 += kR) {
@@ -388,7 +390,7 @@ __device__ void final_select(uint2* region, const int* cnt, Anchor anc, int k, i
       for (int u = 0; u < kR; ++u)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          xv[u][i] = r0 + u < c[i] ? __ldcs(&mine_col[(int64_t)(r0 + u) * 128 + 32 * i].x) : 0u;
+          xv[u][i] = r0 + u < c[i] ? __ldcg(&mine_col[(int64_t)(r0 + u) * 128 + 32 * i].x) : 0u;
 #pragma unroll
       for (int u = 0; u < kR; ++u)
 #pragma unroll
