@@ -377,6 +377,14 @@ def split_prof(prof):
     return kern, cnt
 
 
+def is_streamed(kernels) -> bool:
+    """Whether a step's routed scoring was the streaming prefill pass: its
+    candidates are selected by the pass after it ("select"); the row-scoring
+    path (decode) takes a row top-k instead.  (A MISA-dagger prefill runs both
+    a selection and the re-rank's row top-k: it is streamed.)"""
+    return "select" in kernels
+
+
 def decode_kbytes(wl):
     """K prefix bytes the decode scorer streams: each group of 256/m queries
     of a sequence reads its longest prefix once (256 B per key)."""
@@ -607,9 +615,7 @@ def measure_config(cfg, args, world, rank, dev, steps, headline, clocks=None):
     p90 = max_over_ranks(step_ms[min(len(step_ms) - 1, (9 * len(step_ms)) // 10)], world)
     kernels = summarise_kernels(kerns, steps)
     k = kernels.get("score", {"ms_per_step": float("nan"), "launches_per_step": 0})
-    # the streaming prefill pass: its candidates are selected by the pass
-    # after it ("select"); decode scores rows and takes the row top-k
-    streamed = "select" in kernels
+    streamed = is_streamed(kernels)
     res = {"workload": bn.workload, "ms_per_step": ms, "latency_ms": ms,
            "value": bn.job_pairs / (ms / 1e3), "unit": UNIT,
            "step_ms_p50": p50, "step_ms_p90": p90, "cuda_graph": bn.use_graph,

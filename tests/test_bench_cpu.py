@@ -147,3 +147,11 @@ def test_roofline_uses_the_burst_peak_for_prefill_and_hbm_for_decode():
     r2 = bench.roofline_of(wl2, 0.01, 1, False, peaks, {}, "none")
     abytes = (1000 + 500) * 256 + 4 * wl2.pairs
     assert r2["bound"] == "hbm" and abs(r2["achieved"] - abytes / 1e-5 / 1e9) < 1e-6
+
+
+def test_streamed_rule_follows_the_selection_pass():
+    # prefill (streaming pass + selection), decode (score rows + row top-k) and
+    # the MISA-dagger prefill (streamed keep, then the re-rank's row top-k)
+    assert bench.is_streamed({"route": 1, "score": 1, "select": 1})
+    assert not bench.is_streamed({"route": 1, "score": 1, "topk": 1})
+    assert bench.is_streamed({"score": 1, "select": 1, "rerank_score": 1, "topk": 1})
