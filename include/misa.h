@@ -239,8 +239,10 @@ int misa_selftest_timeout(int32_t wait_ms, misa_stream_t stream);
 /* Tracing.  While enabled (on != 0), every kernel the library launches from
  * the calling host thread is bracketed by CUDA events recorded on its launch
  * stream.  misa_profile_collect synchronises those events and returns, per
- * kernel name (names: max_kernels x 32 chars), the summed device time in
- * milliseconds and the launch count, then clears the record.  Returns the
+ * traced name (names: max_kernels x 32 chars), the summed device time in
+ * milliseconds and the number of kernels launched under it (one per name,
+ * except "plan_groups" for plans of more than 256 query groups: a scan and a
+ * fill), then clears the record.  Returns the
  * number of kernel names (at most max_kernels) or a negative MISA_ERR code.
  * Names starting with '#' are counters, not kernels (time 0, the count in
  * `launches`): "#rescan_queries" sums, over the streaming top-k calls traced,

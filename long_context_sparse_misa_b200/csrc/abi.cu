@@ -108,6 +108,7 @@ namespace {
 struct ProfRecord {
   const char* name;
   cudaEvent_t start, stop;
+  int kernels;  // kernels launched inside the scope
 };
 thread_local bool t_prof_on = false;
 thread_local std::vector<ProfRecord> t_prof;       // recorded, not yet collected
@@ -142,7 +143,7 @@ int num_sms() {
 
 ProfScope::ProfScope(const char* name, cudaStream_t s) : slot(-1), st(s) {
   if (!t_prof_on) return;
-  ProfRecord r{name, take_event(), take_event()};
+  ProfRecord r{name, take_event(), take_event(), 1};
   if (!r.start || !r.stop) return;
   cudaEventRecord(r.start, st);
   t_prof.push_back(r);
@@ -151,6 +152,12 @@ ProfScope::ProfScope(const char* name, cudaStream_t s) : slot(-1), st(s) {
 
 ProfScope::~ProfScope() {
   if (slot >= 0) cudaEventRecord(t_prof[slot].stop, st);
+}
+
+// A scope that launches more than one kernel adds the others to its record
+// (the innermost open scope is the last one recorded).
+void prof_add_kernels(int n) {
+  if (t_prof_on && !t_prof.empty()) t_prof.back().kernels += n;
 }
 
 void prof_count(const char* name, const int* dev_count, cudaStream_t st) {
@@ -615,10 +622,10 @@ int misa_profile_collect(int32_t max_kernels, char* names, double* total_ms, int
     auto it = acc.find(r.name);
     if (it == acc.end()) {
       order.push_back(r.name);
-      acc[r.name] = {ms, 1};
+      acc[r.name] = {ms, r.kernels};
     } else {
       it->second.first += ms;
-      it->second.second += 1;
+      it->second.second += r.kernels;
     }
     t_free_events.push_back(r.start);
     t_free_events.push_back(r.stop);
